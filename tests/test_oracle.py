@@ -1,0 +1,266 @@
+"""Pins of the fp64 oracle against facts fixed by the pages and by mathematics.
+
+None of these retypes the oracle's formula: each check is a closed form, a
+hand-derived value, an invariant, an independent library routine, or the
+pages' own blockwise algorithm agreeing with the definition.  The last group
+plants known mistakes in the oracle (on the CPU) and shows that the pins catch
+them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import attention_fp64 as oracle_mod
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_derived_cases.json")
+TIGHT = 1e-12
+
+
+def rand(shape, seed, amp=1.0):
+    return amp * np.random.default_rng(seed).standard_normal(shape)
+
+
+def sdpa_f64(q, k, v, scale, causal):
+    """torch's float64 CPU scaled_dot_product_attention (an independent library
+    routine) with K/V heads expanded for GQA and the bottom-right causal mask
+    passed explicitly; LSE from torch.logsumexp."""
+    q, k, v = (torch.from_numpy(np.ascontiguousarray(x)).double() for x in (q, k, v))
+    rep = q.shape[1] // k.shape[1]
+    k = k.repeat_interleave(rep, dim=1)
+    v = v.repeat_interleave(rep, dim=1)
+    Nq, Nk = q.shape[2], k.shape[2]
+    mask = None
+    if causal:
+        mask = torch.ones(Nq, Nk, dtype=torch.bool).tril(diagonal=Nk - Nq)
+    o = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=mask, scale=scale)
+    s = scale * (q @ k.transpose(-1, -2))
+    if mask is not None:
+        s = s.masked_fill(~mask, float("-inf"))
+    return o.numpy(), torch.logsumexp(s, dim=-1).numpy()
+
+
+# ---------------------------------------------------------------- golden cases
+def load_golden():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+@pytest.mark.parametrize("case", load_golden()["cases"], ids=lambda c: c["name"])
+def test_hand_derived_prefill_cases(case):
+    q, k, v = (np.array(case[n], dtype=np.float64) for n in ("q", "k", "v"))
+    O, LSE = oracle.attention(q, k, v, case["scale"], case["causal"])
+    np.testing.assert_allclose(O, np.array(case["O"]), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(LSE, np.array(case["LSE"]), rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("case", load_golden()["decode_cases"], ids=lambda c: c["name"])
+def test_hand_derived_decode_cases(case):
+    O, LSE = oracle.decode_paged(np.array(case["q"]), np.array(case["kcache"]),
+                                 np.array(case["vcache"]), np.array(case["block_table"]),
+                                 np.array(case["seq_lens"]), case["scale"], case["page_size"])
+    np.testing.assert_allclose(O, np.array(case["O"]), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(LSE, np.array(case["LSE"]), rtol=0, atol=1e-13)
+
+
+# ---------------------------------------------------------------- closed forms
+@pytest.mark.parametrize("causal", [False, True])
+def test_zero_query_gives_mean_of_visible_values(causal):
+    B, Hq, Hkv, Nq, Nk, D = 2, 4, 2, 5, 9, 6
+    q = np.zeros((B, Hq, Nq, D))
+    k, v = rand((B, Hkv, Nk, D), 1), rand((B, Hkv, Nk, D), 2)
+    O, LSE = oracle.attention(q, k, v, 0.3, causal)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // (Hq // Hkv)
+            for i in range(Nq):
+                n = i + (Nk - Nq) + 1 if causal else Nk
+                np.testing.assert_allclose(O[b, h, i], v[b, g, :n].mean(axis=0), atol=TIGHT)
+                assert abs(LSE[b, h, i] - math.log(n)) < TIGHT
+
+
+def test_single_dominant_key_selects_its_value():
+    Nk, D = 16, 8
+    q = rand((1, 1, 1, D), 3)
+    k = rand((1, 1, Nk, D), 4) * 0.01
+    j = 11
+    k[0, 0, j] = 60.0 * q[0, 0, 0] / np.dot(q[0, 0, 0], q[0, 0, 0])   # score 60 vs ~0
+    v = rand((1, 1, Nk, D), 5)
+    O, LSE = oracle.attention(q, k, v, 1.0, False)
+    bound = Nk * math.exp(-59.0) * np.abs(v).max() + 1e-12     # weight off key j <= Nk e^-59
+    np.testing.assert_allclose(O[0, 0, 0], v[0, 0, j], atol=bound)
+    assert abs(LSE[0, 0, 0] - 60.0) < 1e-12 + Nk * math.exp(-59)
+
+
+def test_causal_first_row_is_first_value():
+    q, k, v = rand((1, 3, 7, 5), 6), rand((1, 3, 7, 5), 7), rand((1, 3, 7, 5), 8)
+    O, LSE = oracle.attention(q, k, v, 0.7, True)
+    np.testing.assert_allclose(O[0, :, 0], v[0, :, 0], atol=TIGHT)
+    np.testing.assert_allclose(LSE[0, :, 0], 0.7 * np.einsum("hd,hd->h", q[0, :, 0], k[0, :, 0]),
+                               atol=TIGHT)
+
+
+def test_single_key_and_constant_values():
+    q, k = rand((2, 2, 4, 3), 9), rand((2, 2, 1, 3), 10)
+    v = rand((2, 2, 1, 3), 11)
+    O, _ = oracle.attention(q, k, v, 1.3, False)
+    np.testing.assert_allclose(O, np.broadcast_to(v, O.shape), atol=TIGHT)
+    c = np.array([0.5, -2.0, 3.25])
+    k2 = rand((2, 2, 6, 3), 12)
+    v2 = np.broadcast_to(c, (2, 2, 6, 3)).copy()
+    O2, _ = oracle.attention(rand((2, 2, 4, 3), 13), k2, v2, 0.9, True)
+    np.testing.assert_allclose(O2, np.broadcast_to(c, O2.shape), atol=TIGHT)
+
+
+def test_fully_masked_row_is_zero_with_minus_inf_lse():
+    s = np.array([[1.0, 2.0], [3.0, 4.0]])
+    p, m, l = oracle.softmax_rows(s, np.array([[True, True], [False, False]]))
+    assert np.all(p[1] == 0) and m[1] == -np.inf and l[1] == 0
+
+
+# ---------------------------------------------------------------- invariants
+def test_softmax_rows_sum_to_one_and_shift_invariance():
+    s = rand((6, 33), 14, amp=20.0)
+    p, m, l = oracle.softmax_rows(s)
+    np.testing.assert_allclose(p.sum(axis=-1), 1.0, atol=TIGHT)
+    delta = rand((6, 1), 15, amp=50.0)
+    p2, m2, l2 = oracle.softmax_rows(s + delta)
+    np.testing.assert_allclose(p2, p, atol=TIGHT)
+    np.testing.assert_allclose(m2, m + delta[:, 0], atol=1e-10)
+    np.testing.assert_allclose(l2, l, rtol=1e-12)
+
+
+def test_joint_key_value_permutation_invariance():
+    q, k, v = rand((1, 2, 5, 4), 16), rand((1, 2, 12, 4), 17), rand((1, 2, 12, 4), 18)
+    perm = np.random.default_rng(19).permutation(12)
+    O1, L1 = oracle.attention(q, k, v, 0.5, False)
+    O2, L2 = oracle.attention(q, k[:, :, perm], v[:, :, perm], 0.5, False)
+    np.testing.assert_allclose(O1, O2, atol=TIGHT)
+    np.testing.assert_allclose(L1, L2, atol=TIGHT)
+
+
+# ---------------------------------------------------------------- library routine
+@pytest.mark.parametrize("Hq,Hkv,Nq,Nk,causal", [(2, 2, 7, 7, False), (4, 1, 9, 9, True),
+                                                  (8, 2, 5, 13, True), (4, 2, 16, 3, False)])
+def test_matches_float64_library_attention(Hq, Hkv, Nq, Nk, causal):
+    q, k, v = rand((2, Hq, Nq, 8), 20), rand((2, Hkv, Nk, 8), 21), rand((2, Hkv, Nk, 8), 22)
+    O, LSE = oracle.attention(q, k, v, 0.35, causal)
+    O_ref, LSE_ref = sdpa_f64(q, k, v, 0.35, causal)
+    np.testing.assert_allclose(O, O_ref, atol=TIGHT)
+    np.testing.assert_allclose(LSE, LSE_ref, atol=TIGHT)
+
+
+def test_rows_variant_matches_library():
+    q, k, v = rand((1, 4, 20, 8), 23), rand((1, 2, 20, 8), 24), rand((1, 2, 20, 8), 25)
+    rows = [(0, 0, 0), (0, 1, 19), (0, 3, 7), (0, 2, 13)]
+    O, LSE = oracle.attention_rows(q, k, v, 0.4, True, rows)
+    O_ref, LSE_ref = sdpa_f64(q, k, v, 0.4, True)
+    for r, (b, h, i) in enumerate(rows):
+        np.testing.assert_allclose(O[r], O_ref[b, h, i], atol=TIGHT)
+        assert abs(LSE[r] - LSE_ref[b, h, i]) < TIGHT
+
+
+# ---------------------------------------------------------------- blockwise = full
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Nq,Nk", [(12, 12), (7, 12)])
+def test_blockwise_equals_definition_for_every_block_size(causal, Nq, Nk):
+    q, k, v = rand((1, 2, Nq, 4), 26), rand((1, 1, Nk, 4), 27), rand((1, 1, Nk, 4), 28)
+    O_ref, L_ref = oracle.attention(q, k, v, 0.8, causal)
+    for Br in range(1, Nq + 1):
+        for Bc in range(1, Nk + 1):
+            O, L = oracle.blockwise_attention(q, k, v, 0.8, causal, Br, Bc)
+            np.testing.assert_allclose(O, O_ref, atol=TIGHT)
+            np.testing.assert_allclose(L, L_ref, atol=TIGHT)
+
+
+# ---------------------------------------------------------------- merge / split-KV
+def test_merge_of_key_chunks_equals_unsplit():
+    q, k, v = rand((1, 4, 3, 8), 29), rand((1, 2, 40, 8), 30), rand((1, 2, 40, 8), 31)
+    O_ref, L_ref = oracle.attention(q, k, v, 0.5, False)
+    cuts = [0, 1, 9, 10, 27, 40]
+    parts = [oracle.attention(q, k[:, :, a:b], v[:, :, a:b], 0.5, False)
+             for a, b in zip(cuts[:-1], cuts[1:])]
+    O, L = oracle.merge_partials([p[0] for p in parts], [p[1] for p in parts])
+    np.testing.assert_allclose(O, O_ref, atol=TIGHT)
+    np.testing.assert_allclose(L, L_ref, atol=TIGHT)
+
+
+def test_merge_closed_forms():
+    o1, o2 = np.array([1.0, 2.0]), np.array([3.0, -2.0])
+    O, L = oracle.merge_partials([o1, o2], [0.7, 0.7])          # equal mass: average
+    np.testing.assert_allclose(O, [2.0, 0.0], atol=TIGHT)
+    assert abs(L - (0.7 + math.log(2))) < TIGHT
+    O, L = oracle.merge_partials([o1, o2], [math.log(3.0), -np.inf])   # empty part: no weight
+    np.testing.assert_allclose(O, o1, atol=TIGHT)
+    assert abs(L - math.log(3.0)) < TIGHT
+
+
+# ---------------------------------------------------------------- paged decode
+def test_decode_matches_definition_on_gathered_cache():
+    rng = np.random.default_rng(32)
+    B, Hq, Hkv, D, ps, pool = 3, 8, 2, 8, 4, 20
+    lens = np.array([1, 9, 13])
+    perm = rng.permutation(pool)
+    table = np.zeros((B, 4), dtype=np.int32)
+    cur = 0
+    for b in range(B):
+        n = -(-lens[b] // ps)
+        table[b, :n] = perm[cur:cur + n]
+        cur += n
+    kc, vc = rand((pool, ps, Hkv, D), 33), rand((pool, ps, Hkv, D), 34)
+    q = rand((B, Hq, D), 35)
+    O, L = oracle.decode_paged(q, kc, vc, table, lens, 0.3, ps)
+    for b in range(B):
+        pages = table[b, :-(-lens[b] // ps)]
+        kk = np.concatenate([kc[p] for p in pages])[:lens[b]]      # [n, Hkv, D]
+        vv = np.concatenate([vc[p] for p in pages])[:lens[b]]
+        o_ref, l_ref = sdpa_f64(q[b][None, :, None, :], kk.transpose(1, 0, 2)[None],
+                                vv.transpose(1, 0, 2)[None], 0.3, False)
+        np.testing.assert_allclose(O[b], o_ref[0, :, 0], atol=TIGHT)
+        np.testing.assert_allclose(L[b], l_ref[0, :, 0], atol=TIGHT)
+
+
+# ---------------------------------------------------------------- planted mistakes
+def test_pins_catch_the_printed_blockwise_update():
+    """The page's update omits L_old; with more than one key block it is wrong."""
+    q, k, v = rand((1, 1, 6, 4), 36), rand((1, 1, 6, 4), 37), rand((1, 1, 6, 4), 38)
+    O_ref, _ = oracle.attention(q, k, v, 1.0, False)
+    O_bug, _ = oracle.blockwise_attention(q, k, v, 1.0, False, 3, 2, keep_page_bug=True)
+    assert np.max(np.abs(O_bug - O_ref)) > 1e-3
+    O_one, _ = oracle.blockwise_attention(q, k, v, 1.0, False, 3, 6, keep_page_bug=True)
+    np.testing.assert_allclose(O_one, O_ref, atol=TIGHT)   # one block: no merge, no bug
+
+
+def test_pins_catch_wrong_gqa_mapping(monkeypatch):
+    q, k, v = rand((1, 4, 5, 4), 39), rand((1, 2, 5, 4), 40), rand((1, 2, 5, 4), 41)
+    monkeypatch.setattr(oracle_mod, "kv_head_of", lambda h, Hq, Hkv: h % Hkv)
+    O_bad, _ = oracle_mod.attention(q, k, v, 0.5, False)
+    O_ref, _ = sdpa_f64(q, k, v, 0.5, False)
+    assert np.max(np.abs(O_bad - O_ref)) > 1e-3
+
+
+def test_pins_catch_top_left_causal_alignment(monkeypatch):
+    q, k, v = rand((1, 1, 4, 4), 42), rand((1, 1, 9, 4), 43), rand((1, 1, 9, 4), 44)
+    monkeypatch.setattr(oracle_mod, "causal_allowed",
+                        lambda Nq, Nk: np.arange(Nk)[None, :] <= np.arange(Nq)[:, None])
+    O_bad, _ = oracle_mod.attention(q, k, v, 0.5, True)
+    O_ref, _ = sdpa_f64(q, k, v, 0.5, True)
+    assert np.max(np.abs(O_bad - O_ref)) > 1e-3
+
+
+def test_pins_catch_missing_normalisation(monkeypatch):
+    """Dropping the division by the row sum changes the golden case's output."""
+    case = load_golden()["cases"][0]
+    q, k, v = (np.array(case[n], dtype=np.float64) for n in ("q", "k", "v"))
+    real = oracle_mod.softmax_rows
+
+    def unnormalised(s, allowed=None):
+        p, m, l = real(s, allowed)
+        return p * l[..., None], m, np.ones_like(l)
+    monkeypatch.setattr(oracle_mod, "softmax_rows", unnormalised)
+    O_bad, _ = oracle_mod.attention(q, k, v, case["scale"], case["causal"])
+    assert np.max(np.abs(O_bad - np.array(case["O"]))) > 1e-3
