@@ -1,0 +1,383 @@
+#!/usr/bin/env python
+"""Benchmark of the exact tiled attention hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+  * prefill: fa_fwd on the Llama-3-8B-shaped GQA causal workload
+    (B=1, Hq=32, Hkv=8, Nq=Nk=8192, D=128, bf16, scale 1/sqrt(128));
+  * decode:  fa_decode_paged on the paged-cache workload (B=64 sequences,
+    Hq=32, Hkv=8, D=128, pages of 16 tokens, lengths U[512, 8192], pool of
+    40000 pages, bf16).
+Each kernel launch is timed with CUDA events on the launching stream; a 256 MiB
+buffer is written before every launch so no launch finds its inputs in L2.
+
+``value`` is prefill TFLOP/s (4*B*Hq*Nq*Nk*D / 2 for causal) summed over ranks
+and divided by the slowest rank's prefill time; the decode KV GB/s is reported
+beside it.  Multi-GPU runs are weak-scaled replicas (each rank runs the same
+per-rank workload on its own inputs; the path has no exchange step).
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
+workloads (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from exact_tiled_attention_40_b200.inputs import (DECODE_CASES, PREFILL_CASES,  # noqa: E402
+                                                  make_decode, make_prefill)
+
+METRIC = "attention TFLOP/s & % BF16 tensor peak (prefill); decode KV GB/s & % HBM peak"
+PREFILL = PREFILL_CASES["gqa_b1_hq32_hkv8_n8192_d128_causal"]
+DECODE = DECODE_CASES["decode_b64_hq32_hkv8_d128_page16"]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLUSH_BYTES = 256 << 20
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash(name: str) -> str:
+    with open(os.path.join(ROOT, "exact_tiled_attention_40_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, source: str):
+    """DRAM bytes per launch recorded from an ncu capture of the current source,
+    or None when no capture matches the source as it is now."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    h = kernel_source_hash(source)
+    for line in open(path):
+        parts = line.split()
+        if len(parts) >= 3 and parts[0] == kernel and parts[1] == h:
+            return float(parts[2])
+    return None
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            cols = [c.strip() for c in line.split(",")]
+            if len(cols) < 8:
+                continue
+            try:
+                sm.append(float(cols[0]))
+                smax = float(cols[1])
+            except ValueError:
+                continue
+            for n, c in zip(names, cols[4:8]):
+                if c.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": ["no samples"]}
+        loaded = sorted(sm)[len(sm) // 4:] or sm       # drop the idle ramp-up samples
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_prefill_sample(heads: int = 8):
+    """fp64 oracle on the first `heads` query heads (and their KV heads) of the
+    prefill workload, full causal rows.  Returns (TFLOP/s, seconds, sample text)."""
+    import oracle
+    q, k, v, _ = make_prefill(PREFILL)
+    g = PREFILL.Hq // PREFILL.Hkv
+    hk = max(1, heads // g)
+    qs = q[:, :heads].float().double().numpy()
+    ks = k[:, :hk].float().double().numpy()
+    vs = v[:, :hk].float().double().numpy()
+    t0 = time.perf_counter()
+    oracle.attention(qs, ks, vs, PREFILL.softmax_scale, True)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * heads * PREFILL.Nq * PREFILL.Nk * PREFILL.D / 2
+    return flops / dt / 1e12, dt, (f"{heads} of {PREFILL.Hq} query heads of "
+                                   f"{PREFILL.name} (full causal rows), fp64")
+
+
+def oracle_decode_sample(seqs: int = 8):
+    import oracle
+    q, kc, vc, table, lens = make_decode(DECODE)
+    kcf, vcf = kc.float().numpy(), vc.float().numpy()
+    t0 = time.perf_counter()
+    oracle.decode_paged(q[:seqs].float().double().numpy(), kcf, vcf, table[:seqs].numpy(),
+                        lens[:seqs].numpy(), DECODE.softmax_scale, DECODE.page_size)
+    dt = time.perf_counter() - t0
+    kv_bytes = int(lens[:seqs].sum()) * DECODE.Hkv * DECODE.D * 2 * 2
+    return kv_bytes / dt / 1e9, dt, f"{seqs} of {DECODE.B} sequences of {DECODE.name}, fp64"
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    vals, dts = [], []
+    for i in range(args.warmup + args.steps):
+        tf, dt, sample = oracle_prefill_sample(heads=1)
+        if i >= args.warmup:
+            vals.append(tf)
+            dts.append(dt)
+    dec_gbs, dec_dt, dec_sample = oracle_decode_sample(seqs=2)
+    value = statistics.median(vals)
+    cores = cpu_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.mean(dts), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": PREFILL.name, "decode_workload": DECODE.name,
+                   "l2": "oracle runs on the host"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "decode": {"value": dec_gbs, "unit": "GB/s", "sample": dec_sample},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    from exact_tiled_attention_40_b200 import fa
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+        pg = torch.distributed.group.WORLD
+
+    def barrier():
+        if pg is not None:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    # ---- inputs: each rank its own replica (seed offset by rank), resident in HBM
+    pcase = dataclasses.replace(PREFILL, seed=PREFILL.seed + 1000 * rank)
+    dcase = dataclasses.replace(DECODE, seed=DECODE.seed + 1000 * rank)
+    q_h, k_h, v_h, _ = make_prefill(pcase)
+    dq_h, kc_h, vc_h, table_h, lens_h = make_decode(dcase)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((pcase.B, pcase.Hq, pcase.Nq), dtype=torch.float32, device=dev)
+    dq, kc, vc = dq_h.to(dev), kc_h.to(dev), vc_h.to(dev)
+    table, lens = table_h.to(dev), lens_h.to(dev)
+    do = torch.empty_like(dq)
+    dlse = torch.empty((dcase.B, dcase.Hq), dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    sum_len = int(lens_h.sum())
+    kv_bytes = sum_len * dcase.Hkv * dcase.D * 2 * 2
+    dec_bytes = kv_bytes + dq.numel() * 2 * 2 + dlse.numel() * 4 + table_h.numel() * 4 \
+        + lens_h.numel() * 4
+
+    def prefill():
+        fa.fa_fwd(q, k, v, o, lse, pcase.B, pcase.Hq, pcase.Hkv, pcase.Nq, pcase.Nk, pcase.D,
+                  pcase.softmax_scale, pcase.causal, stream=sp)
+
+    def decode():
+        fa.fa_decode_paged(dq, kc, vc, table, lens, do, dcase.B, dcase.Hq, dcase.Hkv, dcase.D,
+                           dcase.page_size, dcase.softmax_scale, table.shape[1], dcase.num_pages,
+                           dlse, stream=sp)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)]
+          for _ in range(args.warmup + args.steps)]
+
+    def step(i):
+        flush.fill_(i & 0xff)
+        ev[i][0].record(stream)
+        prefill()
+        ev[i][1].record(stream)
+        flush.fill_((i + 1) & 0xff)
+        ev[i][2].record(stream)
+        decode()
+        ev[i][3].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    barrier()
+    sampler = ClockSampler(local)
+    with sampler:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        barrier()
+        t0.record(stream)
+        for i in range(args.warmup, args.warmup + args.steps):
+            step(i)
+        t1.record(stream)
+        barrier()
+    assert fa.device_status() == 0, fa.last_error()
+    total_ms = t0.elapsed_time(t1)
+    pre_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.warmup, args.warmup + args.steps)]
+    dec_ms = [ev[i][2].elapsed_time(ev[i][3]) for i in range(args.warmup, args.warmup + args.steps)]
+
+    # ---- end to end through the C ABI with pinned host buffers
+    qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+    op = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    lp = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h2d = (qp.numel() + kp.numel() + vp.numel()) * 2
+    d2h = op.numel() * 2 + lp.numel() * 4
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(i & 0xff)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        q.copy_(qp, non_blocking=True)
+        k.copy_(kp, non_blocking=True)
+        v.copy_(vp, non_blocking=True)
+        prefill()
+        op.copy_(o, non_blocking=True)
+        lp.copy_(lse, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b))
+
+    # ---- reduce over ranks (max time, summed work)
+    sums = torch.tensor([sum(pre_ms), sum(dec_ms), total_ms, sum(e2e_ms)], dtype=torch.float64,
+                        device=dev)
+    if pg is not None:
+        torch.distributed.all_reduce(sums, op=torch.distributed.ReduceOp.MAX)
+    pre_max, dec_max, total_max, e2e_max = sums.tolist()
+    K = args.steps
+    value = world * K * pcase.flops / (pre_max * 1e-3) / 1e12
+    dec_gbs = world * K * kv_bytes / (dec_max * 1e-3) / 1e9
+    e2e_val = world * K * pcase.flops / (e2e_max * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    avg_pre_s = statistics.mean(pre_ms) * 1e-3
+    avg_dec_s = statistics.mean(dec_ms) * 1e-3
+    achieved = pcase.flops / avg_pre_s / 1e12
+    dec_achieved = dec_bytes / avg_dec_s / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": total_max / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": pcase.name, "decode_workload": dcase.name,
+                   "B": pcase.B, "Hq": pcase.Hq, "Hkv": pcase.Hkv, "seq_len": pcase.Nq,
+                   "head_dim": pcase.D, "causal": pcase.causal,
+                   "decode_sum_len_per_rank": sum_len,
+                   "l2": f"{FLUSH_BYTES >> 20} MiB buffer written before every launch",
+                   "parallelism": f"replicas x{world} (weak scaling, no collective)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                     "traffic": recorded_traffic("fa_fwd_kernel", "fa_fwd_sm100.cu"),
+                     "kernel": "fa_fwd_kernel<128,bf16>", "peak_source": f"{peak_src} burst bf16",
+                     "frac_of_nominal_2250": achieved / 2250.0},
+        "decode": {"value": dec_gbs, "unit": "GB/s", "kv_bytes_per_step": kv_bytes,
+                   "roofline": {"bound": "hbm", "achieved": dec_achieved, "peak": peaks["hbm_gbs"],
+                                "unit": "GB/s", "frac": dec_achieved / peaks["hbm_gbs"],
+                                "traffic": recorded_traffic("fa_decode_split_kernel",
+                                                            "fa_decode_sm100.cu"),
+                                "peak_source": f"{peak_src} copy bandwidth",
+                                "frac_of_nominal_8000": dec_achieved / 8000.0},
+                   "ms_per_launch": statistics.mean(dec_ms)},
+        "prefill_ms_per_launch": statistics.mean(pre_ms),
+        "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "what": "prefill through fa_fwd with pinned host "
+                "q,k,v copied in and o,lse copied out inside the timed region"},
+        "gpu_launches": 3 * K,
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, dt, sample = oracle_prefill_sample(heads=8)
+        line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cpu_threads(),
+                                "kind": "oracle", "sample": sample, "seconds": dt}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

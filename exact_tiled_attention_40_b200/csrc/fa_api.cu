@@ -1,0 +1,175 @@
+// C-ABI entry points: argument validation on the host, error reporting and the
+// per-device error word.  Every compute step runs in the kernels of
+// fa_fwd_sm100.cu and fa_decode_sm100.cu; there is no host fallback.
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "fa_internal.h"
+#include "ptx_sm100.cuh"
+#include "../../include/fa.h"
+
+namespace fa {
+
+namespace {
+thread_local char g_msg[512] = "";
+__device__ int g_error_word;   // see kErrTimeout / kErrBadIndex
+std::mutex g_err_mu;
+int* g_err_ptr[64] = {};
+}  // namespace
+
+int set_error(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int* device_error_word(int device) {
+  if (device < 0 || device >= 64) return nullptr;
+  std::lock_guard<std::mutex> g(g_err_mu);
+  if (!g_err_ptr[device]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
+    g_err_ptr[device] = static_cast<int*>(p);
+  }
+  return g_err_ptr[device];
+}
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The current device must be an sm_100 part; its ordinal is returned in *dev.
+int current_sm100(int* dev) {
+  int d = -1;
+  cudaError_t e = cudaGetDevice(&d);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return set_error(FA_ERR_NO_DEVICE, "no CUDA device: %s", cudaGetErrorString(e));
+  }
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, d);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, d);
+  if (major != 10 || minor != 0)
+    return set_error(FA_ERR_NO_DEVICE, "device %d is sm_%d%d; this library is built for sm_100a",
+                     d, major, minor);
+  *dev = d;
+  return FA_OK;
+}
+
+int validate_fwd(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv,
+                 int Nq, int Nk, int D, float scale, int causal) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || Nq < 0 || Nk < 0)
+    return set_error(FA_ERR_INVALID_ARG, "negative size");
+  if (!(std::isfinite(scale) && scale > 0.f))
+    return set_error(FA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (D != 64 && D != 128)
+    return set_error(FA_ERR_UNSUPPORTED, "head dimension %d is not supported (64 or 128)", D);
+  if (B == 0 || Hq == 0 || Nq == 0) return FA_OK;
+  if (Hkv <= 0 || Hq % Hkv != 0)
+    return set_error(FA_ERR_INVALID_ARG, "Hq (%d) must be a positive multiple of Hkv (%d)", Hq,
+                     Hkv);
+  if (causal && Nq > Nk)
+    return set_error(FA_ERR_INVALID_ARG, "causal attention needs Nq <= Nk (got %d > %d)", Nq, Nk);
+  if (!q || !o || (Nk > 0 && (!k || !v))) return set_error(FA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(o) || (Nk > 0 && (!aligned16(k) || !aligned16(v))))
+    return set_error(FA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (static_cast<long long>(B) * Hq > 0x7fffffffLL || static_cast<long long>(B) * Hkv > 0x7fffffffLL)
+    return set_error(FA_ERR_UNSUPPORTED, "B * H too large");
+  return FA_OK;
+}
+
+int fwd_common(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+               int Hkv, int Nq, int Nk, int D, float scale, int causal, cudaStream_t stream,
+               bool bf16) {
+  int rc = validate_fwd(q, k, v, o, B, Hq, Hkv, Nq, Nk, D, scale, causal);
+  if (rc != FA_OK) return rc;
+  if (B == 0 || Hq == 0 || Nq == 0) return FA_OK;
+  int dev;
+  if ((rc = current_sm100(&dev)) != FA_OK) return rc;
+  return launch_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, bf16, stream, dev);
+}
+
+}  // namespace
+}  // namespace fa
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+           int Hkv, int Nq, int Nk, int D, float scale, int causal, fa_stream_t stream) {
+  return fa::fwd_common(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal,
+                        reinterpret_cast<cudaStream_t>(stream), true);
+}
+
+int fa_fwd_fp16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                int Hkv, int Nq, int Nk, int D, float scale, int causal, fa_stream_t stream) {
+  return fa::fwd_common(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal,
+                        reinterpret_cast<cudaStream_t>(stream), false);
+}
+
+int fa_decode_paged(const void* q, const void* kcache, const void* vcache,
+                    const int32_t* block_table, const int32_t* seq_lens, void* o, int B, int Hq,
+                    int Hkv, int D, int page_size, float scale, fa_stream_t stream,
+                    int max_pages_per_seq, int num_pages, float* lse) {
+  using namespace fa;
+  if (B < 0 || Hq < 0 || Hkv < 0 || max_pages_per_seq < 0 || num_pages < 0)
+    return set_error(FA_ERR_INVALID_ARG, "negative size");
+  if (!(std::isfinite(scale) && scale > 0.f))
+    return set_error(FA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (D != 128) return set_error(FA_ERR_UNSUPPORTED, "decode supports D == 128 only (got %d)", D);
+  if (page_size != 16)
+    return set_error(FA_ERR_UNSUPPORTED, "decode supports page_size == 16 only (got %d)",
+                     page_size);
+  if (B == 0 || Hq == 0) return FA_OK;
+  if (Hkv <= 0 || Hq % Hkv != 0)
+    return set_error(FA_ERR_INVALID_ARG, "Hq (%d) must be a positive multiple of Hkv (%d)", Hq,
+                     Hkv);
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8)
+    return set_error(FA_ERR_UNSUPPORTED, "decode supports Hq/Hkv in {1,2,4,8} (got %d)", G);
+  if (max_pages_per_seq <= 0 || num_pages <= 0)
+    return set_error(FA_ERR_INVALID_ARG, "max_pages_per_seq and num_pages must be positive");
+  if (!q || !kcache || !vcache || !block_table || !seq_lens || !o)
+    return set_error(FA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o))
+    return set_error(FA_ERR_INVALID_ARG, "q, caches and o must be 16-byte aligned");
+  if (static_cast<long long>(max_pages_per_seq) * 16 > 0x7fffffffLL)
+    return set_error(FA_ERR_INVALID_ARG, "max_pages_per_seq too large");
+  int dev, rc;
+  if ((rc = current_sm100(&dev)) != FA_OK) return rc;
+  return launch_decode(q, kcache, vcache, block_table, seq_lens, o, lse, B, Hq, Hkv, D, page_size,
+                       scale, max_pages_per_seq, num_pages, reinterpret_cast<cudaStream_t>(stream),
+                       dev);
+}
+
+const char* fa_last_error_string(void) { return fa::g_msg; }
+
+int fa_device_status(void) {
+  using namespace fa;
+  int dev;
+  int rc = current_sm100(&dev);
+  if (rc != FA_OK) return rc;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return set_error(FA_ERR_CUDA, "device: %s", cudaGetErrorString(e));
+  int word = 0;
+  e = cudaMemcpyFromSymbol(&word, g_error_word, sizeof(int));
+  if (e != cudaSuccess) return set_error(FA_ERR_CUDA, "error word: %s", cudaGetErrorString(e));
+  if (word == 0) return FA_OK;
+  const int zero = 0;
+  cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int));
+  if (word & kErrTimeout)
+    return set_error(FA_ERR_DEVICE_TIMEOUT, "a bounded in-kernel wait ran out (word 0x%x)", word);
+  return set_error(FA_ERR_DEVICE_INDEX, "out-of-range block-table entry or length (word 0x%x)",
+                   word);
+}
+
+void fa_release(void) { fa::release_decode_resources(); }
+
+int fa_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,479 @@
+// Exact tiled attention forward for sm_100a.
+//
+// Method: the blockwise online-softmax algorithm of unite.ai, "Flash Attention:
+// Revolutionizing Transformer Efficiency", section "Implementation Details"
+// (query blocks outer, key/value blocks inner, running row max M and row sum L),
+// with the softmax decomposition and merge of section "The Mathematics of
+// Flash Attention".  O is kept unnormalised and divided by L once at the end.
+//
+// One CTA owns two 128-row query tiles (Q0, Q1) of one (batch, head) and streams
+// the 128-key K/V tiles of the matching KV head (GQA, devhandbook example 5)
+// through a ring of shared-memory slots.  Warp roles (320 threads):
+//   warps 0-3  softmax warpgroup for Q0   (thread r owns query row r = TMEM lane r)
+//   warps 4-7  softmax warpgroup for Q1
+//   warp  8    TMA producer: Q tiles once, then K_j, V_j into the slot ring
+//   warp  9    TMEM allocator and single-thread tcgen05 MMA issuer
+// Tensor memory (512 columns x 128 lanes, fp32):
+//   [  0,128) S0 = Q0 K^T  (its first 64 columns are reused for P0 as bf16 pairs)
+//   [128,256) S1 = Q1 K^T  (P1 likewise)
+//   [256,256+D) O0,  [256+D,256+2D) O1  -- the running unnormalised outputs
+// Per key tile j the MMA thread issues, in order: PV0_j, S0_{j+1}, PV1_j, S1_{j+1}.
+// tcgen05 operations of one thread execute in issue order, so S_{j+1} never
+// overwrites P_j before PV_j has read it, and the commit that publishes S_{j+1}
+// also guarantees PV_j finished -- the softmax warpgroup may then rescale O in
+// place before it releases P_{j+1}.
+// The rescale is lazy: a row's reference maximum only moves when the new tile
+// maximum exceeds it by more than 2^8, so P stays <= 256 and O is rescaled only
+// on those rare tiles.  Exactness is unaffected: O and L share the reference.
+#include <cfloat>
+#include <cstdio>
+#include <mutex>
+
+#include "fa_internal.h"
+#include "ptx_sm100.cuh"
+#include "../../include/fa.h"
+
+namespace fa {
+namespace {
+
+constexpr int kBM = 128;       // query rows per tile = TMEM lanes
+constexpr int kBN = 128;       // keys per tile
+constexpr float kTau = 8.0f;   // lazy-rescale threshold (log2 units)
+constexpr int kThreads = 320;
+
+template <int D>
+struct FwdLayout {
+  static constexpr int kChunks = D / 64;              // 128-byte swizzle atoms along D
+  static constexpr int kChunkBytes = kBM * 128;       // one atom column of a 128-row tile
+  static constexpr int kTileBytes = kBM * D * 2;      // a 128-row tile of Q, K or V
+  static constexpr int kSlots = D == 128 ? 4 : 8;     // K/V ring slots
+  static constexpr int kQOff = 0;
+  static constexpr int kKVOff = 2 * kTileBytes;
+  static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
+  static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 2 + 2 + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + slack for 1024-byte alignment
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+struct FwdParams {
+  void* o;
+  float* lse;
+  int B, Hq, Hkv, Nq, Nk;
+  int num_mpairs;
+  int causal;
+  float scale_log2;   // scale * log2(e)
+  int* err;
+  uint64_t timeout_ns;
+};
+
+__device__ __forceinline__ int kv_tiles_for(int first_row, const FwdParams& p) {
+  if (first_row >= p.Nq) return 0;
+  const int nk_tiles = (p.Nk + kBN - 1) / kBN;
+  if (!p.causal) return nk_tiles;
+  const int last_row = min(first_row + kBM - 1, p.Nq - 1);
+  const int max_key = last_row + (p.Nk - p.Nq);
+  return min(nk_tiles, max_key / kBN + 1);
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using L = FwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+
+  // ---- work item: (batch, head, pair of query tiles); causal: heaviest first
+  const int BH = p.B * p.Hq;
+  const int mrev = blockIdx.x / BH;
+  const int bh = blockIdx.x - mrev * BH;
+  const int mpair = p.causal ? (p.num_mpairs - 1 - mrev) : mrev;
+  const int b = bh / p.Hq;
+  const int h = bh - b * p.Hq;
+  const int hkv = h / (p.Hq / p.Hkv);
+  const int q_row0 = mpair * 2 * kBM;
+  int n_kv[2];
+  n_kv[0] = kv_tiles_for(q_row0, p);
+  n_kv[1] = kv_tiles_for(q_row0 + kBM, p);
+  const int n_max = max(n_kv[0], n_kv[1]);
+
+  auto bar = [&](int i) -> uint32_t { return sbase + L::kBarOff + 8 * i; };
+  auto q_full = [&](int t) { return bar(t); };
+  auto kv_full = [&](int s) { return bar(2 + s); };
+  auto kv_empty = [&](int s) { return bar(2 + L::kSlots + s); };
+  auto s_full = [&](int t) { return bar(2 + 2 * L::kSlots + t); };
+  auto p_full = [&](int t) { return bar(4 + 2 * L::kSlots + t); };
+  auto o_full = [&](int t) { return bar(6 + 2 * L::kSlots + t); };
+  const uint32_t mma_done = bar(8 + 2 * L::kSlots);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+
+  if (tid == 0) {
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(q_full(t), 1);
+      mbar_init(s_full(t), 1);
+      mbar_init(p_full(t), kBM);
+      mbar_init(o_full(t), 1);
+    }
+    for (int s = 0; s < L::kSlots; ++s) {
+      mbar_init(kv_full(s), 1);
+      mbar_init(kv_empty(s), 1);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && n_max > 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      for (int t = 0; t < 2; ++t) {
+        if (n_kv[t] == 0) continue;
+        mbar_arrive_expect_tx(q_full(t), L::kTileBytes);
+        const uint32_t dst = sbase + L::kQOff + t * L::kTileBytes;
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_3d(dst + c * L::kChunkBytes, &tmQ, q_full(t), c * 64, q_row0 + t * kBM, bh);
+      }
+      const int kv_z = b * p.Hkv + hkv;
+      int issued = 0;
+      for (int j = 0; j < n_max; ++j) {
+        bool ok = true;
+        for (int w = 0; w < 2; ++w) {
+          const int pos = 2 * j + w;
+          const int slot = pos % L::kSlots;
+          const uint32_t ph = (pos / L::kSlots) & 1;
+          if (!mbar_wait(kv_empty(slot), ph ^ 1, abort_flag, p.err, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(kv_full(slot), L::kTileBytes);
+          const uint32_t dst = sbase + L::kKVOff + slot * L::kTileBytes;
+          const void* tm = w ? static_cast<const void*>(&tmV) : static_cast<const void*>(&tmK);
+          for (int c = 0; c < L::kChunks; ++c)
+            tma_load_3d(dst + c * L::kChunkBytes, tm, kv_full(slot), c * 64, j * kBN, kv_z);
+          ++issued;
+        }
+        if (!ok) break;
+      }
+      // Every issued copy must land before the CTA may exit (also on abort).
+      volatile int no_abort = 0;
+      for (int t = 0; t < 2; ++t)
+        if (n_kv[t] > 0) mbar_wait(q_full(t), 0, &no_abort, p.err, p.timeout_ns);
+      for (int s = 0; s < L::kSlots && s < issued; ++s) {
+        const int last = s + ((issued - 1 - s) / L::kSlots) * L::kSlots;
+        mbar_wait(kv_full(s), (last / L::kSlots) & 1, &no_abort, p.err, p.timeout_ns);
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_max > 0) {
+      constexpr uint32_t idesc_s = idesc_f16(kBM, kBN, BF16, false);
+      constexpr uint32_t idesc_pv = idesc_f16(kBM, D, BF16, true);
+      bool ok = true;
+      for (int t = 0; t < 2 && ok; ++t)
+        if (n_kv[t] > 0) ok = mbar_wait(q_full(t), 0, abort_flag, p.err, p.timeout_ns);
+      auto slot_of = [&](int pos) { return pos % L::kSlots; };
+      auto phase_of = [&](int pos) { return static_cast<uint32_t>((pos / L::kSlots) & 1); };
+      // S_t = Q_t K^T : M=128, N=128, K=D in steps of 16 (32 bytes inside a swizzle atom)
+      auto issue_s = [&](int t, int slot) {
+        const uint32_t qa = sbase + L::kQOff + t * L::kTileBytes;
+        const uint32_t kb = sbase + L::kKVOff + slot * L::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
+          mma_ss(tmem + t * 128, smem_desc_sw128(qa + off, 16, 1024),
+                 smem_desc_sw128(kb + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(s_full(t));
+      };
+      // O_t += P_t V : A = P from TMEM (bf16 pairs), B = V tile, MN-major (D contiguous)
+      auto issue_pv = [&](int t, int slot, bool accumulate) {
+        const uint32_t vb = sbase + L::kKVOff + slot * L::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8,
+                 smem_desc_sw128(vb + kk * 16 * 128, L::kChunkBytes, 1024), idesc_pv,
+                 (accumulate || kk > 0) ? 1u : 0u);
+        }
+      };
+      if (ok) ok = mbar_wait(kv_full(slot_of(0)), phase_of(0), abort_flag, p.err, p.timeout_ns);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < 2; ++t)
+          if (n_kv[t] > 0) issue_s(t, slot_of(0));
+        tc_commit(kv_empty(slot_of(0)));
+      }
+      for (int j = 0; j < n_max && ok; ++j) {
+        const int vpos = 2 * j + 1;
+        const int kpos = 2 * j + 2;
+        const bool has_next = j + 1 < n_max;
+        ok = mbar_wait(kv_full(slot_of(vpos)), phase_of(vpos), abort_flag, p.err, p.timeout_ns);
+        if (ok && has_next)
+          ok = mbar_wait(kv_full(slot_of(kpos)), phase_of(kpos), abort_flag, p.err, p.timeout_ns);
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j >= n_kv[t]) continue;
+          ok = mbar_wait(p_full(t), j & 1, abort_flag, p.err, p.timeout_ns);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(t, slot_of(vpos), j > 0);
+          if (j + 1 < n_kv[t])
+            issue_s(t, slot_of(kpos));
+          else
+            tc_commit(o_full(t));
+        }
+        if (!ok) break;
+        tc_commit(kv_empty(slot_of(vpos)));
+        if (has_next) tc_commit(kv_empty(slot_of(kpos)));
+      }
+      // All issued MMAs must complete before TMEM is released (also on abort).
+      tc_commit(mma_done);
+      volatile int no_abort = 0;
+      mbar_wait(mma_done, 0, &no_abort, p.err, p.timeout_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int t = warp >> 2;
+    const int r = tid & 127;
+    const int row = q_row0 + t * kBM + r;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + t * 128;
+    const uint32_t tO = tmem + lane_base + 256 + t * D;
+    const int n = n_kv[t];
+    const size_t row_index = static_cast<size_t>(bh) * p.Nq + row;
+    using Out = uint16_t;
+    Out* o_row = reinterpret_cast<Out*>(p.o) + row_index * D;
+    if (n == 0) {
+      if (row < p.Nq && q_row0 + t * kBM < p.Nq) {   // only reached when Nk == 0
+        uint4 z = make_uint4(0, 0, 0, 0);
+        for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(o_row)[c] = z;
+        if (p.lse) p.lse[row_index] = -INFINITY;
+      }
+    } else {
+      float m_used = -INFINITY;
+      float l = 0.f;
+      const int off = p.Nk - p.Nq;
+      const int tile_first = q_row0 + t * kBM;
+      bool ok = true;
+      for (int j = 0; j < n; ++j) {
+        if (!mbar_wait(s_full(t), j & 1, abort_flag, p.err, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t s[128];
+        tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+        tmem_wait_ld();
+        const int kbase = j * kBN;
+        const bool need_mask =
+            (kbase + kBN > p.Nk) || (p.causal && kbase + kBN - 1 > tile_first + off);
+        if (need_mask) {
+          int lim = p.Nk - 1 - kbase;                       // last visible column
+          if (p.causal) lim = min(lim, row + off - kbase);
+#pragma unroll
+          for (int e = 0; e < 128; ++e)
+            if (e > lim) s[e] = __float_as_uint(-INFINITY);
+        }
+        float mx = __uint_as_float(s[0]);
+#pragma unroll
+        for (int e = 1; e < 128; ++e) mx = fmaxf(mx, __uint_as_float(s[e]));
+        const float m_tile = mx * p.scale_log2;
+        if (m_tile > m_used + kTau) {
+          const float alpha = ex2(m_used - m_tile);   // 0 on the first visible tile
+          if (j > 0) {
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t ov[32];
+              tmem_ld32(tO + 32 * c, ov);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+              tmem_st32(tO + 32 * c, ov);
+            }
+          }
+          l *= alpha;
+          m_used = m_tile;
+        }
+        const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
+        float sum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = ex2(fmaf(__uint_as_float(s[32 * c + 2 * e]), p.scale_log2, neg_m));
+            const float p1 =
+                ex2(fmaf(__uint_as_float(s[32 * c + 2 * e + 1]), p.scale_log2, neg_m));
+            sum += p0 + p1;
+            pk[e] = BF16 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
+          }
+          tmem_st16(tS + 16 * c, pk);
+        }
+        l += sum;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full(t));
+      }
+      if (ok && mbar_wait(o_full(t), 0, abort_flag, p.err, p.timeout_ns)) {
+        tc_fence_after();
+        const float inv_l = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(tO + 32 * c, ov);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float a = __uint_as_float(ov[2 * e]) * inv_l;
+            const float bb = __uint_as_float(ov[2 * e + 1]) * inv_l;
+            pk[e] = BF16 ? pack_bf16x2(a, bb) : pack_f16x2(a, bb);
+          }
+          if (row < p.Nq) {
+            uint4* dst = reinterpret_cast<uint4*>(o_row + 32 * c);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
+        }
+        if (p.lse && row < p.Nq)
+          p.lse[row_index] = l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) ==
+            cudaSuccess &&
+        qres == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 3-D map over a contiguous [Z, N, D] tensor of 16-bit elements with a
+// 64 x 128 x 1 box and 128-byte swizzle (one swizzle atom column per box).
+int encode_3d(CUtensorMap* m, const void* base, bool bf16, int D, int N, int Z) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return set_error(FA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(Z)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                           static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(D) * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                   const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return set_error(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", int(r));
+  return FA_OK;
+}
+
+template <int D, bool BF16>
+int launch_typed(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                 int Hkv, int Nq, int Nk, float scale, int causal, cudaStream_t stream,
+                 int device) {
+  using L = FwdLayout<D>;
+  static bool attr_done[64] = {};
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> g(mu);
+    if (device < 0 || device >= 64) return set_error(FA_ERR_CUDA, "device ordinal out of range");
+    if (!attr_done[device]) {
+      cudaError_t e = cudaFuncSetAttribute(fa_fwd_kernel<D, BF16>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           L::kSmemBytes);
+      if (e != cudaSuccess)
+        return set_error(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+      attr_done[device] = true;
+    }
+  }
+  CUtensorMap tq, tk, tv;
+  int rc;
+  // Nk == 0 never reaches a TMA load; give the maps a valid extent anyway.
+  if ((rc = encode_3d(&tq, q, BF16, D, Nq, B * Hq)) != FA_OK) return rc;
+  if ((rc = encode_3d(&tk, k, BF16, D, Nk > 0 ? Nk : 1, B * Hkv)) != FA_OK) return rc;
+  if ((rc = encode_3d(&tv, v, BF16, D, Nk > 0 ? Nk : 1, B * Hkv)) != FA_OK) return rc;
+  FwdParams prm;
+  prm.o = o;
+  prm.lse = lse;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.Nq = Nq;
+  prm.Nk = Nk;
+  prm.num_mpairs = (Nq + 2 * kBM - 1) / (2 * kBM);
+  prm.causal = causal ? 1 : 0;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.err = device_error_word(device);
+  prm.timeout_ns = kWaitLimitNs;
+  if (!prm.err) return set_error(FA_ERR_CUDA, "device error word unavailable");
+  const long long grid = static_cast<long long>(prm.num_mpairs) * B * Hq;
+  if (grid > 0x7fffffffLL) return set_error(FA_ERR_UNSUPPORTED, "grid too large");
+  fa_fwd_kernel<D, BF16><<<static_cast<unsigned>(grid), kThreads, L::kSmemBytes, stream>>>(
+      tq, tk, tv, prm);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(FA_ERR_CUDA, "fa_fwd launch: %s", cudaGetErrorString(e));
+  return FA_OK;
+}
+
+}  // namespace
+
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+               int Hkv, int Nq, int Nk, int D, float scale, int causal, bool bf16,
+               cudaStream_t stream, int device) {
+  if (D == 128)
+    return bf16 ? launch_typed<128, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal,
+                                          stream, device)
+                : launch_typed<128, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal,
+                                           stream, device);
+  if (D == 64)
+    return bf16 ? launch_typed<64, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal,
+                                         stream, device)
+                : launch_typed<64, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal,
+                                          stream, device);
+  return set_error(FA_ERR_UNSUPPORTED, "head dimension %d is not supported (64 or 128)", D);
+}
+
+}  // namespace fa

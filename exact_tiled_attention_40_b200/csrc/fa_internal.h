@@ -1,0 +1,33 @@
+// Declarations shared by the library's translation units (not part of the ABI).
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace fa {
+
+// Record a message for fa_last_error_string() (thread-local) and return `code`.
+int set_error(int code, const char* fmt, ...);
+
+// Device pointer of the per-device error word that kernels set on a bounded
+// wait running out or on an out-of-range index read from device memory.
+int* device_error_word(int device);
+
+// Wall-time limit of every bounded wait inside a kernel.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+// Forward prefill launcher (validated arguments).  bf16 selects bf16 inputs,
+// otherwise fp16.  Returns an FA_* status.
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+               int Hkv, int Nq, int Nk, int D, float scale, int causal, bool bf16,
+               cudaStream_t stream, int device);
+
+// Split-KV paged decode launcher (validated arguments).
+int launch_decode(const void* q, const void* kcache, const void* vcache, const int32_t* block_table,
+                  const int32_t* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int D,
+                  int page_size, float scale, int max_pages_per_seq, int num_pages,
+                  cudaStream_t stream, int device);
+
+// Release cached per-device resources owned by the decode path.
+void release_decode_resources();
+
+}  // namespace fa

@@ -1,0 +1,143 @@
+"""Thin Python binding of the C ABI in include/fa.h (argument marshalling only).
+
+Every function forwards device pointers, sizes and the current CUDA stream to
+``libfa_sm100.so``; all arithmetic runs in that library's sm_100a kernels.
+There is no fallback: if the library or a CUDA device is missing, calls raise.
+PyTorch is used for device memory and streams only.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libfa_sm100.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "fa.h")
+
+FA_OK = 0
+STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_CUDA",
+          4: "FA_ERR_DEVICE_TIMEOUT", 5: "FA_ERR_DEVICE_INDEX", 6: "FA_ERR_NO_DEVICE"}
+
+_lib = None
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_SIGS = {
+    "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_fwd_fp16": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _I, _I, _P]),
+    "fa_last_error_string": (ctypes.c_char_p, []),
+    "fa_device_status": (_I, []),
+    "fa_release": (None, []),
+    "fa_version": (_I, []),
+}
+
+
+class FAError(RuntimeError):
+    def __init__(self, code: int, where: str, msg: str):
+        super().__init__(f"{where}: {STATUS.get(code, code)}: {msg}")
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    """Load the shared library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise FAError(-1, "load", f"{LIB_PATH} is missing; run "
+                          "`python -m exact_tiled_attention_40_b200.build`")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(l, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = l
+    return _lib
+
+
+def header_symbols() -> list[str]:
+    """Names of the functions declared in include/fa.h."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(fa_\w+)\s*\(", text, re.M)))
+
+
+def _check(code: int, where: str):
+    if code != FA_OK:
+        raise FAError(code, where, lib().fa_last_error_string().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, stream=None):
+    """Raw call of the C entry point (bf16 or fp16 chosen from q's dtype)."""
+    fn = lib().fa_fwd if q.dtype == torch.bfloat16 else lib().fa_fwd_fp16
+    s = _stream(q.device) if stream is None else ctypes.c_void_p(stream)
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, D,
+              float(scale), int(bool(causal)), s), "fa_fwd")
+
+
+def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None = None,
+              causal: bool = False, return_lse: bool = True):
+    """O, LSE for q [B,Hq,Nq,D] and k, v [B,Hkv,Nk,D] (bf16 or fp16, contiguous CUDA)."""
+    if not (q.is_cuda and k.is_cuda and v.is_cuda):
+        raise FAError(1, "attention", "tensors must live on a CUDA device")
+    if q.dtype not in (torch.bfloat16, torch.float16) or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise FAError(1, "attention", "q, k, v must share dtype bf16 or fp16")
+    q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    B, Hq, Nq, D = q.shape
+    _, Hkv, Nk, _ = k.shape
+    if scale is None:
+        scale = D ** -0.5
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device) if return_lse else None
+    fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal)
+    return o, lse
+
+
+def fa_decode_paged(q, kcache, vcache, block_table, seq_lens, o, B, Hq, Hkv, D, page_size, scale,
+                    max_pages_per_seq, num_pages, lse=None, stream=None):
+    """Raw call of the C entry point."""
+    s = _stream(q.device) if stream is None else ctypes.c_void_p(stream)
+    _check(lib().fa_decode_paged(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(block_table),
+                                 _ptr(seq_lens), _ptr(o), B, Hq, Hkv, D, page_size, float(scale),
+                                 s, max_pages_per_seq, num_pages, _ptr(lse)), "fa_decode_paged")
+
+
+def decode_paged(q, kcache, vcache, block_table, seq_lens, scale=None, return_lse=True):
+    """O [B,Hq,D] (and LSE [B,Hq]) for one query token per sequence over a paged cache."""
+    B, Hq, D = q.shape
+    num_pages, page_size, Hkv, _ = kcache.shape
+    if scale is None:
+        scale = D ** -0.5
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise FAError(1, "decode_paged", "block_table and seq_lens must be int32")
+    block_table = block_table.contiguous()
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device) if return_lse else None
+    fa_decode_paged(q.contiguous(), kcache.contiguous(), vcache.contiguous(), block_table,
+                    seq_lens.contiguous(), o, B, Hq, Hkv, D, page_size, scale,
+                    block_table.shape[1], num_pages, lse)
+    return o, lse
+
+
+def device_status() -> int:
+    """Synchronise and read/clear the device error word (FA_* code)."""
+    return lib().fa_device_status()
+
+
+def last_error() -> str:
+    return lib().fa_last_error_string().decode()
+
+
+def release():
+    lib().fa_release()

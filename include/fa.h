@@ -1,0 +1,125 @@
+/*
+ * Exact tiled attention for NVIDIA B200 (sm_100a): C ABI.
+ *
+ * The library computes exact scaled-dot-product attention
+ *     O = softmax(scale * Q K^T [+ causal mask]) V
+ * tile by tile with the online-softmax decomposition (running row maximum and
+ * row sum, old partial results rescaled by exp(m_old - m_new)), so the
+ * Nq x Nk score matrix never reaches device memory.  Sources:
+ *   - unite.ai, "Flash Attention: Revolutionizing Transformer Efficiency":
+ *     opening listing standard_attention (the definition), section "The
+ *     Mathematics of Flash Attention" (softmax decomposition and merge) and
+ *     section "Implementation Details" (the blockwise loop with running M, L).
+ *   - devhandbook.co.kr, "Flash Attention 2 ... PyTorch native": example 1
+ *     ([B, H, L, D] tensors), example 3 (is_causal), example 5 (GQA, 32 query
+ *     heads over 8 KV heads), section 4 (head dimension 64 or 128).
+ *   - cabseo.com, "Advanced techniques for enhancing LLM throughput": sections
+ *     "Memory requirements" (KV cache), "Autoregressive and memory-bound
+ *     operations" (one query token per decode step) and "Paged attention".
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, 16-byte
+ *     aligned, contiguous row-major.  The library keeps no reference to them
+ *     after the call returns.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and never synchronise the device.
+ *   - Return value: FA_OK (0) or an FA_ERR_* code; fa_last_error_string()
+ *     then describes the failure (per calling thread).  Argument errors are
+ *     detected on the host before anything is launched.
+ *   - Faults found inside a kernel (a bounded wait that ran out, an out-of-range
+ *     block-table entry or sequence length) do not trap: the kernel skips the
+ *     bad work and sets a per-device error word that fa_device_status() reads.
+ *   - There is no CPU fallback: without a usable sm_100 device the calls fail.
+ */
+#ifndef EXACT_TILED_ATTENTION_FA_H
+#define EXACT_TILED_ATTENTION_FA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* fa_stream_t; /* identical to cudaStream_t */
+
+enum fa_status {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,    /* null pointer, bad size, misaligned pointer, bad scale */
+  FA_ERR_UNSUPPORTED = 2,    /* valid but not implemented (head dim, page size, group size) */
+  FA_ERR_CUDA = 3,           /* a CUDA runtime call or kernel launch failed */
+  FA_ERR_DEVICE_TIMEOUT = 4, /* fa_device_status(): a bounded in-kernel wait ran out */
+  FA_ERR_DEVICE_INDEX = 5,   /* fa_device_status(): a block-table entry or length was out of range */
+  FA_ERR_NO_DEVICE = 6       /* no sm_100 device is current */
+};
+
+/*
+ * Prefill / full attention, bf16 inputs and output.
+ *
+ * Computes O = softmax(scale * Q K^T [+ causal]) V and LSE per query row.
+ *   q   [B, Hq,  Nq, D] bf16          k, v [B, Hkv, Nk, D] bf16
+ *   o   [B, Hq,  Nq, D] bf16 (written)
+ *   lse [B, Hq,  Nq]    fp32 (written; may be NULL): natural log of the row
+ *       sum of exp(scale * q.k) over the visible keys.
+ * GQA: query head h reads KV head h / (Hq / Hkv); Hq must be a multiple of Hkv.
+ * causal != 0: query i sees key j iff j <= i + (Nk - Nq) (bottom-right
+ *   alignment; query i sees keys 0..i when Nq == Nk); requires Nq <= Nk.
+ * D must be 64 or 128.  scale must be finite and > 0 (the pages use 1/sqrt(D)).
+ * B, Hq or Nq equal to 0 is a no-op.  Nk == 0 (non-causal) writes O = 0 and
+ * LSE = -inf.
+ * Device memory touched: exactly q, k, v (read) and o, lse (written); no
+ * workspace is allocated.
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+           int Hkv, int Nq, int Nk, int D, float scale, int causal, fa_stream_t stream);
+
+/* Same as fa_fwd with fp16 q, k, v and o (fp32 LSE). */
+int fa_fwd_fp16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                int Hkv, int Nq, int Nk, int D, float scale, int causal, fa_stream_t stream);
+
+/*
+ * Decode over a paged KV cache: one new query token per sequence attends over
+ * all of that sequence's cached keys and values (no mask beyond its length).
+ *   q           [B, Hq, D] bf16
+ *   kcache      [num_pages, page_size, Hkv, D] bf16  (token slot t of a page
+ *   vcache      [num_pages, page_size, Hkv, D] bf16   holds all Hkv heads)
+ *   block_table [B, max_pages_per_seq] int32: page ids of sequence b in token
+ *               order; token t lives in page block_table[b][t / page_size],
+ *               slot t % page_size.  Entries past the sequence are not read.
+ *   seq_lens    [B] int32, 0 <= seq_lens[b] <= max_pages_per_seq * page_size
+ *   o           [B, Hq, D] bf16 (written)
+ *   lse         [B, Hq] fp32 (written; may be NULL)
+ * Supported: D == 128, page_size == 16, Hq / Hkv in {1, 2, 4, 8, 16}.
+ * num_pages bounds every block-table entry (0 <= id < num_pages); entries out
+ * of range are skipped and flagged in the device error word.
+ * A sequence of length 0 gets O = 0 and LSE = -inf.
+ * Work is split over key chunks; partial results are merged by their LSE.
+ * The partials live in a stream-ordered workspace taken from a library-owned
+ * memory pool on `stream` and returned to it on `stream` (no device sync);
+ * fa_release() frees the pool.
+ */
+int fa_decode_paged(const void* q, const void* kcache, const void* vcache,
+                    const int32_t* block_table, const int32_t* seq_lens, void* o, int B, int Hq,
+                    int Hkv, int D, int page_size, float scale, fa_stream_t stream,
+                    int max_pages_per_seq, int num_pages, float* lse);
+
+/* Description of the last error returned on this thread ("" if none). */
+const char* fa_last_error_string(void);
+
+/*
+ * Synchronises the current device, then reads and clears its device error
+ * word.  Returns FA_OK, FA_ERR_DEVICE_TIMEOUT, FA_ERR_DEVICE_INDEX or
+ * FA_ERR_CUDA.
+ */
+int fa_device_status(void);
+
+/* Frees the library's cached device resources (decode workspace pools). */
+void fa_release(void);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_TILED_ATTENTION_FA_H */

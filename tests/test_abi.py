@@ -1,0 +1,82 @@
+"""The C-ABI library loads, exports every declared entry point, and validates
+arguments on the host (no GPU needed: nothing here launches a kernel)."""
+import ctypes
+
+import pytest
+import torch
+
+from exact_tiled_attention_40_b200 import fa
+
+E = {v: k for k, v in fa.STATUS.items()}
+FAKE = 0x10000   # 16-byte aligned fake device address; validation never dereferences it
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return fa.lib()
+
+
+def test_every_header_symbol_is_exported(lib):
+    names = fa.header_symbols()
+    assert set(names) >= {"fa_fwd", "fa_fwd_fp16", "fa_decode_paged", "fa_last_error_string",
+                          "fa_device_status", "fa_release", "fa_version"}
+    for n in names:
+        assert hasattr(lib, n), n
+    assert lib.fa_version() >= 100
+
+
+def fwd(lib, B=1, Hq=2, Hkv=1, Nq=8, Nk=8, D=64, scale=0.125, causal=0, q=FAKE, o=FAKE,
+        k=FAKE, v=FAKE):
+    return lib.fa_fwd(q, k, v, o, None, B, Hq, Hkv, Nq, Nk, D, scale, causal, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=-1), "FA_ERR_INVALID_ARG"),
+    (dict(D=96), "FA_ERR_UNSUPPORTED"),
+    (dict(Hq=3, Hkv=2), "FA_ERR_INVALID_ARG"),
+    (dict(Hkv=0), "FA_ERR_INVALID_ARG"),
+    (dict(causal=1, Nq=9, Nk=8), "FA_ERR_INVALID_ARG"),
+    (dict(scale=0.0), "FA_ERR_INVALID_ARG"),
+    (dict(scale=float("nan")), "FA_ERR_INVALID_ARG"),
+    (dict(scale=-1.0), "FA_ERR_INVALID_ARG"),
+    (dict(q=0), "FA_ERR_INVALID_ARG"),
+    (dict(k=0), "FA_ERR_INVALID_ARG"),
+    (dict(o=FAKE + 8), "FA_ERR_INVALID_ARG"),
+])
+def test_fwd_rejects_bad_arguments_on_the_host(lib, kw, code):
+    assert fwd(lib, **kw) == E[code]
+    assert lib.fa_last_error_string().decode() != ""
+
+
+def test_fwd_empty_problem_is_a_noop(lib):
+    assert fwd(lib, B=0) == 0
+    assert fwd(lib, Nq=0) == 0
+    assert fwd(lib, Hq=0) == 0
+
+
+def dec(lib, B=2, Hq=8, Hkv=2, D=128, page=16, scale=0.1, maxp=4, npages=10, ptr=FAKE):
+    return lib.fa_decode_paged(ptr, ptr, ptr, ptr, ptr, ptr, B, Hq, Hkv, D, page, scale, None,
+                               maxp, npages, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(D=64), "FA_ERR_UNSUPPORTED"),
+    (dict(page=32), "FA_ERR_UNSUPPORTED"),
+    (dict(Hq=32, Hkv=1), "FA_ERR_UNSUPPORTED"),
+    (dict(Hq=6, Hkv=4), "FA_ERR_INVALID_ARG"),
+    (dict(maxp=0), "FA_ERR_INVALID_ARG"),
+    (dict(npages=-1), "FA_ERR_INVALID_ARG"),
+    (dict(ptr=0), "FA_ERR_INVALID_ARG"),
+    (dict(ptr=FAKE + 4), "FA_ERR_INVALID_ARG"),
+    (dict(scale=0.0), "FA_ERR_INVALID_ARG"),
+])
+def test_decode_rejects_bad_arguments_on_the_host(lib, kw, code):
+    assert dec(lib, **kw) == E[code]
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_valid_call_without_a_device_fails_loudly(lib):
+    assert fwd(lib) == E["FA_ERR_NO_DEVICE"]
+    assert dec(lib) == E["FA_ERR_NO_DEVICE"]
+    with pytest.raises(fa.FAError):
+        fa._check(fwd(lib), "fa_fwd")
