@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + t * 128;
     const uint32_t tO = tmem + lane_base + 256 + t * D;
-    const int n = n_kv[t];
+    const int n = t ? n_kv[1] : n_kv[0];
     const size_t row_index = static_cast<size_t>(bh) * p.Nq + row;
     using Out = uint16_t;
     Out* o_row = reinterpret_cast<Out*>(p.o) + row_index * D;
@@ -272,7 +272,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tile_first = q_row0 + t * kBM;
       bool ok = true;
       for (int j = 0; j < n; ++j) {
-        if (!mbar_wait(s_full(t), j & 1, abort_flag, p.err, p.timeout_ns)) {
+        // tcgen05.ld/st/wait are warp-collective: every branch around them is
+        // made warp-uniform, also on the abort path.
+        const bool got = mbar_wait(s_full(t), j & 1, abort_flag, p.err, p.timeout_ns);
+        if (!__all_sync(0xffffffffu, got)) {
           ok = false;
           break;
         }
@@ -297,21 +300,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int e = 1; e < 128; ++e) mx = fmaxf(mx, __uint_as_float(s[e]));
         const float m_tile = mx * p.scale_log2;
-        if (m_tile > m_used + kTau) {
-          const float alpha = ex2(m_used - m_tile);   // 0 on the first visible tile
-          if (j > 0) {
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t ov[32];
-              tmem_ld32(tO + 32 * c, ov);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-              tmem_st32(tO + 32 * c, ov);
-            }
-          }
+        const bool move = m_tile > m_used + kTau;
+        float alpha = 1.f;
+        if (move) {
+          alpha = ex2(m_used - m_tile);   // 0 on the first visible tile
           l *= alpha;
           m_used = m_tile;
+        }
+        // Rescale O rows whose reference moved; the whole warp takes part in
+        // the TMEM round trip, rows that did not move keep alpha = 1.
+        if (j > 0 && __any_sync(0xffffffffu, move)) {
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(tO + 32 * c, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st32(tO + 32 * c, ov);
+          }
         }
         const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
         float sum = 0.f;
@@ -333,7 +340,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(p_full(t));
       }
-      if (ok && mbar_wait(o_full(t), 0, abort_flag, p.err, p.timeout_ns)) {
+      const bool fin = ok && mbar_wait(o_full(t), 0, abort_flag, p.err, p.timeout_ns);
+      if (__all_sync(0xffffffffu, fin)) {
         tc_fence_after();
         const float inv_l = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
@@ -431,10 +439,14 @@ int launch_typed(const void* q, const void* k, const void* v, void* o, float* ls
   }
   CUtensorMap tq, tk, tv;
   int rc;
-  // Nk == 0 never reaches a TMA load; give the maps a valid extent anyway.
   if ((rc = encode_3d(&tq, q, BF16, D, Nq, B * Hq)) != FA_OK) return rc;
-  if ((rc = encode_3d(&tk, k, BF16, D, Nk > 0 ? Nk : 1, B * Hkv)) != FA_OK) return rc;
-  if ((rc = encode_3d(&tv, v, BF16, D, Nk > 0 ? Nk : 1, B * Hkv)) != FA_OK) return rc;
+  if (Nk > 0) {
+    if ((rc = encode_3d(&tk, k, BF16, D, Nk, B * Hkv)) != FA_OK) return rc;
+    if ((rc = encode_3d(&tv, v, BF16, D, Nk, B * Hkv)) != FA_OK) return rc;
+  } else {
+    tk = tq;   // no key tile exists, so these maps are never read
+    tv = tq;
+  }
   FwdParams prm;
   prm.o = o;
   prm.lse = lse;
