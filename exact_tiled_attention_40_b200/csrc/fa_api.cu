@@ -147,6 +147,43 @@ int fa_decode_paged(const void* q, const void* kcache, const void* vcache,
                        dev);
 }
 
+int fa_decode_paged_noalloc(const void* q, const void* kcache, const void* vcache,
+                            const int32_t* block_table, const int32_t* seq_lens, void* o, int B,
+                            int Hq, int Hkv, int D, int page_size, float scale, fa_stream_t stream,
+                            int max_pages_per_seq, int num_pages, float* lse) {
+  using namespace fa;
+  if (B < 0 || Hq < 0 || Hkv < 0 || max_pages_per_seq < 0 || num_pages < 0)
+    return set_error(FA_ERR_INVALID_ARG, "negative size");
+  if (!(std::isfinite(scale) && scale > 0.f))
+    return set_error(FA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (D != 128) return set_error(FA_ERR_UNSUPPORTED, "decode supports D == 128 only (got %d)", D);
+  if (page_size != 16)
+    return set_error(FA_ERR_UNSUPPORTED, "decode supports page_size == 16 only (got %d)",
+                     page_size);
+  if (B == 0 || Hq == 0) return FA_OK;
+  if (Hkv <= 0 || Hq % Hkv != 0)
+    return set_error(FA_ERR_INVALID_ARG, "Hq (%d) must be a positive multiple of Hkv (%d)", Hq,
+                     Hkv);
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8)
+    return set_error(FA_ERR_UNSUPPORTED, "decode supports Hq/Hkv in {1,2,4,8} (got %d)", G);
+  if (max_pages_per_seq <= 0 || num_pages <= 0)
+    return set_error(FA_ERR_INVALID_ARG, "max_pages_per_seq and num_pages must be positive");
+  if (!q || !kcache || !vcache || !block_table || !seq_lens || !o)
+    return set_error(FA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o))
+    return set_error(FA_ERR_INVALID_ARG, "q, caches and o must be 16-byte aligned");
+  if (static_cast<long long>(max_pages_per_seq) * 16 > 0x7fffffffLL)
+    return set_error(FA_ERR_INVALID_ARG, "max_pages_per_seq too large");
+  int pps, nsplit, dev, rc;
+  // The scratch bound is checked before the device is touched.
+  if ((rc = plan_decode_noalloc(B, Hq, max_pages_per_seq, &pps, &nsplit)) != FA_OK) return rc;
+  if ((rc = current_sm100(&dev)) != FA_OK) return rc;
+  return launch_decode_noalloc(q, kcache, vcache, block_table, seq_lens, o, lse, B, Hq, Hkv,
+                               max_pages_per_seq, num_pages, scale,
+                               reinterpret_cast<cudaStream_t>(stream), dev);
+}
+
 const char* fa_last_error_string(void) { return fa::g_msg; }
 
 int fa_device_status(void) {

@@ -392,3 +392,116 @@ void release_decode_resources() {
 }
 
 }  // namespace fa
+
+// ---------------------------------------------------------------- no-allocation variant
+//
+// Same split and combine kernels as launch_decode, but the chunk partials live
+// in a fixed array compiled into this library instead of memory obtained at
+// call time, for callers that cannot allocate device memory during a decode
+// step.  The array is part of the library's device image: every GPU on which
+// the library's kernels are loaded holds these bytes until the process exits.
+// Every call shares it and it keeps the previous call's contents; nothing in it
+// has to start at zero, because the merge only reads chunk results written
+// earlier in the same call.  Two calls whose kernels overlap on the GPU (for
+// example on two streams) use the same bytes and race.
+namespace fa {
+
+static __device__ __align__(256) float g_decode_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+namespace {
+std::mutex g_scratch_mu;
+float* g_scratch_ptr[64] = {};
+
+// Device address of g_decode_scratch on `device` (which must be current).  In
+// host code the array's name is only a host-side stand-in; the address a kernel
+// may use comes from cudaGetSymbolAddress, looked up once per device.
+int scratch_address(int device, float** out) {
+  if (device < 0 || device >= 64) return set_error(FA_ERR_CUDA, "device ordinal out of range");
+  std::lock_guard<std::mutex> g(g_scratch_mu);
+  if (!g_scratch_ptr[device]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return set_error(FA_ERR_CUDA, "cudaGetSymbolAddress(decode scratch): %s",
+                       cudaGetErrorString(e));
+    g_scratch_ptr[device] = static_cast<float*>(p);
+  }
+  *out = g_scratch_ptr[device];
+  return FA_OK;
+}
+}  // namespace
+
+int plan_decode_noalloc(int B, int Hq, int max_pages_per_seq, int* pps_out, int* nsplit_out) {
+  // Start from the split size launch_decode would use and widen the splits
+  // until the partials fit the fixed scratch array.
+  long long want = (static_cast<long long>(B) * max_pages_per_seq + 2047) / 2048;
+  long long pps = 4;
+  while (pps < want && pps < 64) pps *= 2;
+  for (;;) {
+    const long long nsplit = (max_pages_per_seq + pps - 1) / pps;
+    const long long bytes = static_cast<long long>(B) * nsplit * Hq * (kDecD + 1) * 4;
+    if (bytes <= static_cast<long long>(kNoAllocScratchBytes)) {
+      *pps_out = static_cast<int>(pps);
+      *nsplit_out = static_cast<int>(nsplit);
+      return FA_OK;
+    }
+    if (nsplit == 1)
+      return set_error(FA_ERR_INVALID_ARG,
+                       "fa_decode_paged_noalloc: B * Hq = %lld needs %lld bytes of scratch even "
+                       "with one chunk per sequence; the fixed scratch holds %zu bytes "
+                       "(B * Hq <= %zu)",
+                       static_cast<long long>(B) * Hq, bytes, kNoAllocScratchBytes,
+                       kNoAllocScratchBytes / ((kDecD + 1) * 4));
+    pps *= 2;
+  }
+}
+
+int launch_decode_noalloc(const void* q, const void* kcache, const void* vcache,
+                          const int32_t* block_table, const int32_t* seq_lens, void* o, float* lse,
+                          int B, int Hq, int Hkv, int max_pages_per_seq, int num_pages,
+                          float scale, cudaStream_t stream, int device) {
+  int pps = 0, nsplit = 0;
+  int rc = plan_decode_noalloc(B, Hq, max_pages_per_seq, &pps, &nsplit);
+  if (rc != FA_OK) return rc;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8)
+    return set_error(FA_ERR_UNSUPPORTED, "decode supports Hq/Hkv in {1,2,4,8} (got %d)", G);
+  float* scratch = nullptr;
+  if ((rc = scratch_address(device, &scratch)) != FA_OK) return rc;
+  DecodeParams prm;
+  prm.q = static_cast<const uint16_t*>(q);
+  prm.kc = static_cast<const uint16_t*>(kcache);
+  prm.vc = static_cast<const uint16_t*>(vcache);
+  prm.block_table = block_table;
+  prm.seq_lens = seq_lens;
+  prm.o = static_cast<uint16_t*>(o);
+  prm.lse = lse;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.max_pages = max_pages_per_seq;
+  prm.num_pages = num_pages;
+  prm.pps = pps;
+  prm.nsplit = nsplit;
+  prm.scale_log2 = scale * kLog2e;
+  prm.err = device_error_word(device);
+  if (!prm.err) return set_error(FA_ERR_CUDA, "device error word unavailable");
+  if (nsplit > 65535 || B > 65535)
+    return set_error(FA_ERR_UNSUPPORTED, "too many sequences or splits for one launch");
+  const size_t n_part = static_cast<size_t>(B) * nsplit * Hq;
+  prm.ws_o = scratch;
+  prm.ws_lse = scratch + n_part * kDecD;
+  switch (G) {
+    case 1: launch_split<1>(prm, stream); break;
+    case 2: launch_split<2>(prm, stream); break;
+    case 4: launch_split<4>(prm, stream); break;
+    default: launch_split<8>(prm, stream); break;
+  }
+  fa_decode_combine_kernel<<<B * Hq, kDecD, 0, stream>>>(prm);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess)
+    return set_error(FA_ERR_CUDA, "decode (no-allocation) launch: %s", cudaGetErrorString(e));
+  return FA_OK;
+}
+
+}  // namespace fa

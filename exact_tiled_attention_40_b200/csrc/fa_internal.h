@@ -1,5 +1,6 @@
 // Declarations shared by the library's translation units (not part of the ABI).
 #pragma once
+#include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -29,5 +30,19 @@ int launch_decode(const void* q, const void* kcache, const void* vcache, const i
 
 // Release cached per-device resources owned by the decode path.
 void release_decode_resources();
+
+// Size of the fixed scratch array used by fa_decode_paged_noalloc.
+constexpr size_t kNoAllocScratchBytes = 16u << 20;   // 16 MiB
+
+// Chunking for fa_decode_paged_noalloc: pages per split and split count such
+// that the partials fit kNoAllocScratchBytes (host only; no device needed).
+int plan_decode_noalloc(int B, int Hq, int max_pages_per_seq, int* pps, int* nsplit);
+
+// Split-KV paged decode whose partials live in the library's fixed scratch
+// array; allocates nothing.  `device` must be the current device.
+int launch_decode_noalloc(const void* q, const void* kcache, const void* vcache,
+                          const int32_t* block_table, const int32_t* seq_lens, void* o, float* lse,
+                          int B, int Hq, int Hkv, int max_pages_per_seq, int num_pages,
+                          float scale, cudaStream_t stream, int device);
 
 }  // namespace fa

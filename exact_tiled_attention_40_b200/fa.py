@@ -30,6 +30,8 @@ _SIGS = {
     "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_fwd_fp16": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _I, _I, _P]),
+    "fa_decode_paged_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _I, _I,
+                                     _P]),
     "fa_last_error_string": (ctypes.c_char_p, []),
     "fa_device_status": (_I, []),
     "fa_release": (None, []),
@@ -128,6 +130,21 @@ def decode_paged(q, kcache, vcache, block_table, seq_lens, scale=None, return_ls
                     seq_lens.contiguous(), o, B, Hq, Hkv, D, page_size, scale,
                     block_table.shape[1], num_pages, lse)
     return o, lse
+
+
+def decode_paged_noalloc(q, kcache, vcache, block_table, seq_lens, o, lse=None, scale=None,
+                         stream=None):
+    """fa_decode_paged_noalloc: same result as decode_paged, written into the
+    caller's o (and lse); the library allocates no device memory for it."""
+    B, Hq, D = q.shape
+    num_pages, page_size, Hkv, _ = kcache.shape
+    if scale is None:
+        scale = D ** -0.5
+    s = _stream(q.device) if stream is None else ctypes.c_void_p(stream)
+    _check(lib().fa_decode_paged_noalloc(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(block_table),
+                                         _ptr(seq_lens), _ptr(o), B, Hq, Hkv, D, page_size,
+                                         float(scale), s, block_table.shape[1], num_pages,
+                                         _ptr(lse)), "fa_decode_paged_noalloc")
 
 
 def device_status() -> int:

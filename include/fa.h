@@ -102,6 +102,40 @@ int fa_decode_paged(const void* q, const void* kcache, const void* vcache,
                     int Hkv, int D, int page_size, float scale, fa_stream_t stream,
                     int max_pages_per_seq, int num_pages, float* lse);
 
+/*
+ * fa_decode_paged without any device-memory allocation.
+ *
+ * The pages have no counterpart of this entry point; it exists for callers that
+ * cannot allocate device memory while they decode.  A serving engine typically
+ * reserves nearly all device memory up front (weights, the KV-cache page pool)
+ * and must not have a decode step fail or stall on an allocation; some
+ * runtimes forbid driver allocations after start-up altogether.
+ * fa_decode_paged takes its chunk workspace from a memory pool on every call;
+ * this variant instead keeps the chunk partials in a fixed 16 MiB array that is
+ * compiled into the library, so it calls no cudaMalloc, cudaFree or pool
+ * allocation.
+ *
+ * Arguments, layouts, supported sizes, outputs and error codes are those of
+ * fa_decode_paged.  Differences:
+ *   - The chunking is widened until the partials fit the array; the result
+ *     agrees with fa_decode_paged within rounding, not bit for bit.
+ *   - Problems whose partials do not fit even with one chunk per sequence
+ *     (B * Hq > 32,513 at D = 128) are rejected with FA_ERR_INVALID_ARG before
+ *     anything touches the device.
+ *   - The array is shared by every call and keeps the previous call's contents
+ *     (nothing in it needs to start at zero).  Calls whose kernels overlap on
+ *     the GPU, e.g. issued on two streams without ordering, race on it.
+ *   - The 16 MiB are held on every GPU on which the library's kernels are
+ *     loaded, until the process exits.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any
+ *     stream capture.
+ */
+int fa_decode_paged_noalloc(const void* q, const void* kcache, const void* vcache,
+                            const int32_t* block_table, const int32_t* seq_lens, void* o, int B,
+                            int Hq, int Hkv, int D, int page_size, float scale,
+                            fa_stream_t stream, int max_pages_per_seq, int num_pages, float* lse);
+
 /* Description of the last error returned on this thread ("" if none). */
 const char* fa_last_error_string(void);
 
