@@ -175,9 +175,9 @@ int fa_decode_paged_noalloc(const void* q, const void* kcache, const void* vcach
     return set_error(FA_ERR_INVALID_ARG, "q, caches and o must be 16-byte aligned");
   if (static_cast<long long>(max_pages_per_seq) * 16 > 0x7fffffffLL)
     return set_error(FA_ERR_INVALID_ARG, "max_pages_per_seq too large");
-  int pps, nsplit, dev, rc;
+  int dev, rc;
   // The scratch bound is checked before the device is touched.
-  if ((rc = plan_decode_noalloc(B, Hq, max_pages_per_seq, &pps, &nsplit)) != FA_OK) return rc;
+  if ((rc = check_decode_noalloc(B, Hq, Hkv, max_pages_per_seq)) != FA_OK) return rc;
   if ((rc = current_sm100(&dev)) != FA_OK) return rc;
   return launch_decode_noalloc(q, kcache, vcache, block_table, seq_lens, o, lse, B, Hq, Hkv,
                                max_pages_per_seq, num_pages, scale,

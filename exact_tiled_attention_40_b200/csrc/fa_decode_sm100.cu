@@ -7,20 +7,30 @@
 // (section "Paged attention"): fixed pages of 16 token slots, each slot holding
 // all KV heads, reached through a per-sequence block table.
 //
-// Kernel 1 (split): grid (split, sequence).  A CTA streams the pages
-// [split * pps, (split + 1) * pps) of one sequence; warp w handles KV head w (and
-// w + 8, ...) together with the Hq/Hkv query heads that share it, so every cache
-// byte is read from HBM exactly once.  Within a warp each half-warp takes one
-// token and each of its 16 lanes a 16-byte slice (8 elements) of the 256-byte
-// head row, so a token row is one coalesced 256-byte read.  Partial dot products
-// for the G query heads are folded across the 16 lanes with a transposing
-// butterfly (each exchange halves the number of live heads), leaving every lane
-// with the full score of one head.  An online softmax (running max, rescale by
-// exp2(m_old - m_new), unnormalised accumulator) runs over the chunk, and the
-// chunk's normalised output and LSE go to a workspace.
-// Kernel 2 (combine): merges a sequence's chunks by their LSE -- the softmax
-// merge of unite.ai, "Flash Attention: Revolutionizing Transformer Efficiency",
-// section "The Mathematics of Flash Attention", formula 2.
+// Within a warp each half-warp takes one token and each of its 16 lanes a
+// 16-byte slice (8 elements) of the 256-byte head row.  Partial dot products for
+// the G query heads that share the KV head are folded across the 16 lanes with a
+// transposing butterfly (each exchange halves the number of live heads), leaving
+// every lane with the full score of one head.  An online softmax (running max,
+// rescale by exp2(m_old - m_new), unnormalised accumulator) runs over the keys,
+// and each chunk's normalised output and LSE go to a workspace that a combine
+// kernel merges by LSE -- the softmax merge of unite.ai, "Flash Attention:
+// Revolutionizing Transformer Efficiency", section "The Mathematics of Flash
+// Attention", formula 2.
+//
+// Two schedules:
+//  * Hkv <= 8 and Hq/Hkv <= 4 (streamed): one persistent CTA per SM.  All sequences' caches form
+//    one list of half-pages (8 token slots: 8 * Hkv * 256 bytes of K and as many
+//    of V, each contiguous in the pool); CTA c takes the equal share
+//    [c*H/C, (c+1)*H/C) of the H half-pages, whatever the sequence lengths.  A
+//    producer warp streams them through a shared-memory ring with bulk async
+//    copies; eight consumer warps (warp g <-> KV head g; 8 lanes per token,
+//    4 tokens per instruction) compute from shared memory and emit one partial
+//    result per (CTA, sequence) segment, stored in
+//    slot c + b (unique: along the list either c or b or both grow by one); a
+//    merge kernel combines each sequence's segments.
+//  * otherwise (direct): grid (chunk, sequence) of fixed page chunks, cache read
+//    straight from HBM with 16-byte non-allocating loads.
 #include <cstdio>
 #include <mutex>
 #include <vector>
@@ -39,6 +49,19 @@ constexpr int kDecThreads = kDecWarps * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.69314718055994530942f;
 
+// streamed schedule
+constexpr int kHalf = 8;                        // token slots per stage
+constexpr int kConsumerWarps = kDecWarps;       // one per KV head (see the stream kernel)
+constexpr int kStreamThreads = 12 * 32;          // 8 consumer warps + a producer warpgroup
+// Register split (setmaxnreg): the producer warpgroup (warps 8-11, one of them
+// working) gives registers to the two consumer warpgroups; 40 x 128 + 224 x 256
+// stays within the 384 x 168 the block is launched with.
+constexpr uint32_t kRegsProducer = 40;
+constexpr uint32_t kRegsConsumer = 224;
+static_assert(kRegsProducer * 128 + kRegsConsumer * 256 <= 384 * 168, "register split");
+constexpr int kMaxStages = 8;
+constexpr int kStreamSmemBudget = 200 * 1024;
+
 struct DecodeParams {
   const uint16_t* q;
   const uint16_t* kc;
@@ -47,9 +70,12 @@ struct DecodeParams {
   const int32_t* seq_lens;
   uint16_t* o;
   float* lse;
-  float* ws_o;     // [B][nsplit][Hq][128] normalised chunk outputs
-  float* ws_lse;   // [B][nsplit][Hq] chunk LSE (natural log)
-  int B, Hq, Hkv, max_pages, num_pages, pps, nsplit;
+  float* ws_o;     // partial outputs, [slot][Hq][128] normalised
+  float* ws_lse;   // partial LSE (natural log), [slot][Hq]
+  int* hb;         // streamed: hb[b] = half-pages before sequence b, hb[B] = total
+  int B, Hq, Hkv, max_pages, num_pages;
+  int pps, nsplit;             // direct schedule
+  int nctas, nstages;          // streamed schedule
   float scale_log2;
   int* err;
 };
@@ -97,6 +123,29 @@ __device__ __forceinline__ float fold_heads(float (&v)[G], int sub) {
   float x = v[0];
 #pragma unroll
   for (int mask = 8 >> LG; mask >= 1; mask >>= 1) x += __shfl_xor_sync(0xffffffffu, x, mask);
+  return x;
+}
+
+// Same fold over the 8 slice lanes of a token (lane bits 0-2 = ls): lane `ls`
+// ends with the total of head ls >> (3 - log2 G).
+template <int G>
+__device__ __forceinline__ float fold_heads8(float (&v)[G], int ls) {
+  constexpr int LG = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3;
+#pragma unroll
+  for (int step = 0; step < LG; ++step) {
+    const int mask = 4 >> step;
+    const bool upper = (ls & mask) != 0;
+    const int n = G >> (step + 1);
+#pragma unroll
+    for (int k = 0; k < n; ++k) {
+      const float keep = upper ? v[k + n] : v[k];
+      const float send = upper ? v[k] : v[k + n];
+      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
+    }
+  }
+  float x = v[0];
+#pragma unroll
+  for (int mask = 4 >> LG; mask >= 1; mask >>= 1) x += __shfl_xor_sync(0xffffffffu, x, mask);
   return x;
 }
 
@@ -252,6 +301,371 @@ __global__ void __launch_bounds__(kDecThreads) fa_decode_split_kernel(const Deco
   }
 }
 
+
+__host__ __device__ constexpr int half_bytes(int Hkv) { return kHalf * Hkv * kDecD * 2; }
+
+// hb[b] = sum over b' < b of ceil(len_b' / 8); hb[B] = total.  One block.
+__global__ void __launch_bounds__(1024) fa_decode_scan_kernel(const DecodeParams p) {
+  __shared__ int warp_sums[32];
+  __shared__ int carry;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < p.B; base += 1024) {
+    const int b = base + threadIdx.x;
+    int v = 0;
+    if (b < p.B) {
+      const int len = checked_len(p, b);
+      if (len < 0)
+        atomicOr(p.err, kErrBadIndex);
+      else
+        v = (len + kHalf - 1) / kHalf;
+    }
+    int x = v;   // inclusive warp scan
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, d);
+      if (lane >= d) x += y;
+    }
+    if (lane == 31) warp_sums[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int w = warp_sums[lane];
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, w, d);
+        if (lane >= d) w += y;
+      }
+      warp_sums[lane] = w;   // inclusive prefix of warp totals
+    }
+    __syncthreads();
+    const int before = carry + (warp > 0 ? warp_sums[warp - 1] : 0) + x - v;
+    if (b < p.B) p.hb[b] = before;
+    __syncthreads();
+    if (threadIdx.x == 1023) carry = before + v;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) p.hb[p.B] = carry;
+}
+
+// CTA c's share of the H half-pages is [c*H/C, (c+1)*H/C); it may be empty.
+__device__ __forceinline__ bool share_nonempty(long long c, long long H, long long C) {
+  return ((c + 1) * H) / C > (c * H) / C;
+}
+// CTA holding half-page x: the largest c with c*H/C <= x.
+__device__ __forceinline__ int cta_of(long long x, long long H, long long C) {
+  return static_cast<int>(((x + 1) * C - 1) / H);
+}
+
+struct StageMeta {
+  int b, hh, flags, len;   // flags: 1 = first of segment, 2 = last of segment, 4 = page valid
+};
+
+template <int G>
+__global__ void __launch_bounds__(kStreamThreads, 1) fa_decode_stream_kernel(const DecodeParams p) {
+  // Consumer warp g owns KV head g and all G query heads that share it, so
+  // every K/V byte is read once from shared memory.
+  constexpr int GW = G;                          // query heads per warp
+  constexpr int LG = GW == 1 ? 0 : GW == 2 ? 1 : GW == 4 ? 2 : 3;
+  constexpr int SHIFT = 3 - LG;                  // slice lane `h << SHIFT` holds head h after the fold
+  constexpr int NQ = kHalf / 4;                  // token quads per stage
+  extern __shared__ __align__(128) uint8_t dsm[];
+  __shared__ __align__(8) uint64_t bars[2 * kMaxStages];
+  __shared__ StageMeta meta[kMaxStages];
+  __shared__ int abort_sm;
+
+  const int c = blockIdx.x;
+  const int C = gridDim.x;
+  const int H = p.hb[p.B];
+  const int x0 = static_cast<int>((static_cast<long long>(c) * H) / C);
+  const int x1 = static_cast<int>((static_cast<long long>(c + 1) * H) / C);
+  const int n = x1 - x0;
+  if (n <= 0) return;                          // the same for every thread of the CTA
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int NS = p.nstages;
+  const int SB = half_bytes(p.Hkv);
+  const uint32_t sbase = smem_u32(dsm);
+  auto full = [&](int st) { return smem_u32(&bars[st]); };
+  auto empty = [&](int st) { return smem_u32(&bars[kMaxStages + st]); };
+  volatile int* abort_flag = &abort_sm;
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < NS; ++st) {
+      mbar_init(full(st), 1);
+      mbar_init(empty(st), kConsumerWarps);
+    }
+    abort_sm = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp >= kConsumerWarps) {
+    regs_dec<kRegsProducer>();
+    if (warp != kConsumerWarps) return;
+    // ---------------------------------------------------------------- producer
+    // The whole warp resolves the next 32 stages (sequence, half-page, page id,
+    // length) with independent loads; lane 0 then issues them in order.
+    int issued = 0;
+    bool ok = true;
+    for (int base = 0; base < n && ok; base += 32) {
+      const int i = base + lane;
+      int bq = 0, hh = 0, page = -1, len = 0, flags = 0;
+      if (i < n) {
+        const int x = x0 + i;
+        int lo = 0, hi = p.B;                  // hb[lo] <= x < hb[hi]
+        while (hi - lo > 1) {
+          const int mid = (lo + hi) >> 1;
+          if (p.hb[mid] <= x) lo = mid; else hi = mid;
+        }
+        bq = lo;
+        const int hb_b = p.hb[bq], hb_n = p.hb[bq + 1];
+        hh = x - hb_b;
+        page = p.block_table[static_cast<size_t>(bq) * p.max_pages + (hh >> 1)];
+        len = p.seq_lens[bq];
+        const bool valid = page >= 0 && page < p.num_pages;
+        flags = ((i == 0 || hh == 0) ? 1 : 0) | ((i == n - 1 || x + 1 == hb_n) ? 2 : 0) |
+                (valid ? 4 : 0);
+      }
+      const int cnt_here = min(32, n - base);
+      for (int k = 0; k < cnt_here; ++k) {
+        const int kb = __shfl_sync(0xffffffffu, bq, k);
+        const int khh = __shfl_sync(0xffffffffu, hh, k);
+        const int kpage = __shfl_sync(0xffffffffu, page, k);
+        const int klen = __shfl_sync(0xffffffffu, len, k);
+        const int kflags = __shfl_sync(0xffffffffu, flags, k);
+        if (lane == 0) {
+          const int ii = base + k;
+          const int st = ii % NS;
+          if (!mbar_wait_sleepy(empty(st), ((ii / NS) & 1) ^ 1, abort_flag, p.err, kWaitLimitNs)) {
+            ok = false;
+          } else {
+            StageMeta md;
+            md.b = kb;
+            md.hh = khh;
+            md.len = klen;
+            md.flags = kflags;
+            meta[st] = md;
+            if (kflags & 4) {
+              const size_t tok0 = static_cast<size_t>(kpage) * kPage + (khh & 1) * kHalf;
+              mbar_arrive_expect_tx(full(st), 2 * SB);
+              bulk_load(sbase + st * 2 * SB, p.kc + tok0 * p.Hkv * kDecD, SB, full(st));
+              bulk_load(sbase + st * 2 * SB + SB, p.vc + tok0 * p.Hkv * kDecD, SB, full(st));
+            } else {
+              atomicOr(p.err, kErrBadIndex);   // consumers skip this stage
+              mbar_arrive(full(st));
+            }
+            ++issued;
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+      }
+    }
+    if (lane == 0) {
+      // copies still in flight must land before the CTA exits
+      volatile int no_abort = 0;
+      for (int i = max(0, issued - NS); i < issued; ++i)
+        mbar_wait(full(i % NS), (i / NS) & 1, &no_abort, p.err, kWaitLimitNs);
+    }
+    return;
+  }
+
+  regs_inc<kRegsConsumer>();
+  // ------------------------------------------------------------------ consumers
+  // Lane = 8 * tq + ls: the warp takes 4 tokens at a time (tq), and each token's
+  // 256-byte head row is split over 8 lanes of 32 bytes (16 elements, ls).
+  const int tq = lane >> 3;
+  const int ls = lane & 7;
+  const int my_head = ls >> SHIFT;
+  const int g = warp;                          // KV head of this warp (idle when g >= Hkv)
+  const bool active = g < p.Hkv;
+  const int hq0 = g * G;
+  const int row_bytes = p.Hkv * kDecD * 2;
+  uint64_t q2[GW][8];
+  uint64_t acc2[GW][8];
+  float m[GW], l[GW];
+  float m_mine = -INFINITY;
+  for (int i = 0; i < n; ++i) {
+    const int st = i % NS;
+    const bool got = mbar_wait(full(st), (i / NS) & 1, abort_flag, p.err, kWaitLimitNs);
+    if (!__all_sync(0xffffffffu, got)) return;
+    const StageMeta md = meta[st];
+    if (active) {
+      if (md.flags & 1) {                      // a new sequence segment begins
+        m_mine = -INFINITY;
+#pragma unroll
+        for (int h = 0; h < GW; ++h) {
+          m[h] = -INFINITY;
+          l[h] = 0.f;
+          const uint4* qp = reinterpret_cast<const uint4*>(
+              p.q + (static_cast<size_t>(md.b) * p.Hq + hq0 + h) * kDecD + ls * 16);
+#pragma unroll
+          for (int v = 0; v < 2; ++v) {
+            const uint4 u = qp[v];
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              acc2[h][4 * v + e] = 0;
+              q2[h][4 * v + e] = f2_pack(__uint_as_float(w[e] << 16) * p.scale_log2,
+                                         __uint_as_float(w[e] & 0xffff0000u) * p.scale_log2);
+            }
+          }
+        }
+      }
+      if (md.flags & 4) {
+        const int ntok = min(kHalf, md.len - md.hh * kHalf);
+        const uint8_t* kst = dsm + st * 2 * SB + (g * kDecD + ls * 16) * 2;
+        const uint8_t* vst = kst + SB;
+        float sc[NQ];
+#pragma unroll
+        for (int qd = 0; qd < NQ; ++qd) {
+          const int t = 4 * qd + tq;
+          const uint4* kp = reinterpret_cast<const uint4*>(kst + t * row_bytes);
+          const uint4 k0 = kp[0], k1 = kp[1];
+          const uint32_t w[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+          float partial[GW];
+#pragma unroll
+          for (int h = 0; h < GW; ++h) {
+            uint64_t a2 = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              a2 = f2_fma(q2[h][e], f2_pack(__uint_as_float(w[e] << 16),
+                                            __uint_as_float(w[e] & 0xffff0000u)), a2);
+            float lo2, hi2;
+            f2_unpack(a2, lo2, hi2);
+            partial[h] = lo2 + hi2;
+          }
+          sc[qd] = fold_heads8<GW>(partial, ls);
+          if (t >= ntok) sc[qd] = -INFINITY;
+        }
+        // stage maximum of this lane's head over its tokens and the other 3 token lanes
+        float mx = sc[0];
+#pragma unroll
+        for (int qd = 1; qd < NQ; ++qd) mx = fmaxf(mx, sc[qd]);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        m_mine = fmaxf(m_mine, mx);
+#pragma unroll
+        for (int h = 0; h < GW; ++h) {
+          const float mh = fmaxf(m[h], __shfl_sync(0xffffffffu, mx, h << SHIFT));
+          const float alpha = (m[h] == -INFINITY) ? 0.f : ex2(m[h] - mh);
+          l[h] *= alpha;
+          const uint64_t a2 = f2_pack(alpha, alpha);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc2[h][e] = f2_mul(acc2[h][e], a2);
+          m[h] = mh;
+        }
+        float pv[NQ];
+        float psum = 0.f;
+#pragma unroll
+        for (int qd = 0; qd < NQ; ++qd) {
+          pv[qd] = (sc[qd] == -INFINITY) ? 0.f : ex2(sc[qd] - m_mine);
+          psum += pv[qd];
+        }
+        psum += __shfl_xor_sync(0xffffffffu, psum, 8);
+        psum += __shfl_xor_sync(0xffffffffu, psum, 16);
+#pragma unroll
+        for (int h = 0; h < GW; ++h) l[h] += __shfl_sync(0xffffffffu, psum, h << SHIFT);
+#pragma unroll
+        for (int qd = 0; qd < NQ; ++qd) {
+          const int t = 4 * qd + tq;
+          // slots past the sequence end hold arbitrary bytes: their V must not
+          // meet a zero weight as NaN * 0
+          uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
+          if (t < ntok) {
+            const uint4* vp = reinterpret_cast<const uint4*>(vst + t * row_bytes);
+            v0 = vp[0];
+            v1 = vp[1];
+          }
+          const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+          for (int h = 0; h < GW; ++h) {
+            // weight of (token t, head h) from the lane of the same token holding head h
+            const float pp = __shfl_sync(0xffffffffu, pv[qd], (tq << 3) | (h << SHIFT));
+            const uint64_t p2 = f2_pack(pp, pp);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              acc2[h][e] = f2_fma(p2, f2_pack(__uint_as_float(w[e] << 16),
+                                              __uint_as_float(w[e] & 0xffff0000u)), acc2[h][e]);
+          }
+        }
+      }
+      if (md.flags & 2) {                      // segment ends: write its partial to slot c + b
+        const size_t base = (static_cast<size_t>(c) + md.b) * p.Hq + hq0;
+#pragma unroll
+        for (int h = 0; h < GW; ++h) {
+          const float inv = l[h] > 0.f ? 1.f / l[h] : 0.f;
+          float4* dst = reinterpret_cast<float4*>(p.ws_o + (base + h) * kDecD + ls * 16);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            float a4[4];
+            f2_unpack(acc2[h][2 * v], a4[0], a4[1]);
+            f2_unpack(acc2[h][2 * v + 1], a4[2], a4[3]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              // the four token lanes accumulated different tokens of the same slice
+              a4[e] += __shfl_xor_sync(0xffffffffu, a4[e], 8);
+              a4[e] += __shfl_xor_sync(0xffffffffu, a4[e], 16);
+            }
+            if (tq == 0) dst[v] = make_float4(a4[0] * inv, a4[1] * inv, a4[2] * inv, a4[3] * inv);
+          }
+          if (tq == 0 && ls == 0)
+            p.ws_lse[base + h] = l[h] > 0.f ? (m[h] + __log2f(l[h])) * kLn2 : -INFINITY;
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty(st));
+  }
+}
+
+// Streamed schedule, merge: one warp per (sequence b, query head h).  The
+// partials of b sit in slots c + b for every CTA c whose non-empty share of the
+// half-page list meets b; they are merged by their LSE (formula 2 of the
+// softmax merge).  Lane i owns output columns [4i, 4i + 4).
+__global__ void __launch_bounds__(128) fa_decode_stream_merge_kernel(const DecodeParams p) {
+  const int wid = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (wid >= p.B * p.Hq) return;
+  const int b = wid / p.Hq;
+  const int h = wid - b * p.Hq;
+  const int xs = p.hb[b], xe = p.hb[b + 1];
+  if (xe <= xs) {                              // no keys (or an invalid length): O = 0, LSE = -inf
+    *reinterpret_cast<uint2*>(p.o + static_cast<size_t>(wid) * kDecD + lane * 4) = make_uint2(0, 0);
+    if (p.lse && lane == 0) p.lse[wid] = -INFINITY;
+    return;
+  }
+  const long long H = p.hb[p.B], C = p.nctas;
+  const int c_first = cta_of(xs, H, C), c_last = cta_of(xe - 1, H, C);
+  // lane-parallel LSE pass over the (few) contributing CTAs
+  float mx = -INFINITY;
+  for (int cc = c_first + lane; cc <= c_last; cc += 32)
+    if (share_nonempty(cc, H, C)) mx = fmaxf(mx, p.ws_lse[(static_cast<size_t>(cc) + b) * p.Hq + h]);
+#pragma unroll
+  for (int d = 16; d >= 1; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
+  float wsum = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (mx > -INFINITY) {
+    for (int cc = c_first; cc <= c_last; ++cc) {
+      if (!share_nonempty(cc, H, C)) continue;
+      const size_t row = (static_cast<size_t>(cc) + b) * p.Hq + h;
+      const float ls = p.ws_lse[row];
+      const float w = (ls == -INFINITY) ? 0.f : ex2((ls - mx) * kLog2e);
+      wsum += w;
+      const float4 v = reinterpret_cast<const float4*>(p.ws_o + row * kDecD)[lane];
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  *reinterpret_cast<uint2*>(p.o + static_cast<size_t>(wid) * kDecD + lane * 4) =
+      make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
+  if (p.lse && lane == 0) p.lse[wid] = wsum > 0.f ? mx + __log2f(wsum) * kLn2 : -INFINITY;
+}
+
 // One CTA of 128 threads per (sequence, query head); thread d owns output column d.
 __global__ void __launch_bounds__(kDecD) fa_decode_combine_kernel(const DecodeParams p) {
   const int bh = blockIdx.x;
@@ -310,10 +724,124 @@ int get_pool(int device, cudaMemPool_t* out) {
   return FA_OK;
 }
 
+int sm_count(int device) {
+  static int cached[64] = {};
+  static std::mutex mu;
+  std::lock_guard<std::mutex> g(mu);
+  if (device < 0 || device >= 64) return 0;
+  if (!cached[device]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) n = 0;
+    cached[device] = n;
+  }
+  return cached[device];
+}
+
+// Launch geometry and workspace size of one decode call.
+struct DecodePlan {
+  bool streamed = false;
+  int pps = 0, nsplit = 0;     // direct schedule
+  int nctas = 0, nstages = 0;  // streamed schedule
+  size_t n_part = 0;           // partial rows (slot x head)
+  size_t bytes = 0;            // workspace bytes
+};
+
+// Direct schedule: pages per chunk so that a full-length batch makes ~2048 CTAs.
+int direct_pps(int B, int max_pages_per_seq) {
+  const long long want = (static_cast<long long>(B) * max_pages_per_seq + 2047) / 2048;
+  int pps = 4;
+  while (pps < want && pps < 64) pps *= 2;
+  return pps;
+}
+
+void finish_plan(DecodePlan& pl, int B, int Hq, int Hkv) {
+  if (pl.streamed) {
+    pl.n_part = (static_cast<size_t>(pl.nctas) + B) * Hq;
+    pl.bytes = pl.n_part * (kDecD + 1) * sizeof(float) + (static_cast<size_t>(B) + 1) * sizeof(int);
+  } else {
+    pl.n_part = static_cast<size_t>(B) * pl.nsplit * Hq;
+    pl.bytes = pl.n_part * (kDecD + 1) * sizeof(float);
+  }
+}
+
+DecodePlan make_plan(int B, int Hq, int Hkv, int max_pages_per_seq, int nsm) {
+  DecodePlan pl;
+  // streamed: one consumer warp per KV head holds the state of G <= 4 query heads
+  pl.streamed = Hkv <= kDecWarps && Hq / Hkv <= 4 && nsm > 0;
+  if (pl.streamed) {
+    pl.nctas = nsm;
+    pl.nstages = kStreamSmemBudget / (2 * half_bytes(Hkv));
+    if (pl.nstages > kMaxStages) pl.nstages = kMaxStages;
+  } else {
+    pl.pps = direct_pps(B, max_pages_per_seq);
+    pl.nsplit = (max_pages_per_seq + pl.pps - 1) / pl.pps;
+  }
+  finish_plan(pl, B, Hq, Hkv);
+  return pl;
+}
+
 template <int G>
-int launch_split(const DecodeParams& prm, cudaStream_t stream) {
-  dim3 grid(prm.nsplit, prm.B);
-  fa_decode_split_kernel<G><<<grid, kDecThreads, 0, stream>>>(prm);
+void launch_kernels(const DecodeParams& prm, const DecodePlan& pl, cudaStream_t stream) {
+  if (G <= 4 && pl.streamed) {
+    const int smem = pl.nstages * 2 * half_bytes(prm.Hkv);
+    static bool attr_done = false;   // the attribute belongs to the function, per process
+    if (!attr_done) {
+      cudaFuncSetAttribute(fa_decode_stream_kernel<(G <= 4 ? G : 4)>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kStreamSmemBudget);
+      attr_done = true;
+    }
+    fa_decode_scan_kernel<<<1, 1024, 0, stream>>>(prm);
+    fa_decode_stream_kernel<(G <= 4 ? G : 4)><<<pl.nctas, kStreamThreads, smem, stream>>>(prm);
+    fa_decode_stream_merge_kernel<<<(prm.B * prm.Hq + 3) / 4, 128, 0, stream>>>(prm);
+  } else {
+    dim3 grid(pl.nsplit, prm.B);
+    fa_decode_split_kernel<G><<<grid, kDecThreads, 0, stream>>>(prm);
+    fa_decode_combine_kernel<<<prm.B * prm.Hq, kDecD, 0, stream>>>(prm);
+  }
+}
+
+// Runs one decode with the given workspace (at least pl.bytes, 256-byte aligned).
+int run_decode(const void* q, const void* kcache, const void* vcache, const int32_t* block_table,
+               const int32_t* seq_lens, void* o, float* lse, int B, int Hq, int Hkv,
+               int max_pages_per_seq, int num_pages, float scale, const DecodePlan& pl, void* ws,
+               cudaStream_t stream, int device) {
+  const int G = Hq / Hkv;
+  DecodeParams prm;
+  prm.q = static_cast<const uint16_t*>(q);
+  prm.kc = static_cast<const uint16_t*>(kcache);
+  prm.vc = static_cast<const uint16_t*>(vcache);
+  prm.block_table = block_table;
+  prm.seq_lens = seq_lens;
+  prm.o = static_cast<uint16_t*>(o);
+  prm.lse = lse;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.max_pages = max_pages_per_seq;
+  prm.num_pages = num_pages;
+  prm.pps = pl.pps;
+  prm.nsplit = pl.nsplit;
+  prm.nctas = pl.nctas;
+  prm.nstages = pl.nstages;
+  prm.scale_log2 = scale * kLog2e;
+  prm.err = device_error_word(device);
+  if (!prm.err) return set_error(FA_ERR_CUDA, "device error word unavailable");
+  if (!pl.streamed && (pl.nsplit > 65535 || B > 65535))
+    return set_error(FA_ERR_UNSUPPORTED, "too many sequences or chunks for one launch");
+  if (static_cast<long long>(B) * Hq > 0x7fffffffLL)
+    return set_error(FA_ERR_UNSUPPORTED, "B * Hq too large");
+  prm.ws_o = static_cast<float*>(ws);
+  prm.ws_lse = prm.ws_o + pl.n_part * kDecD;
+  prm.hb = reinterpret_cast<int*>(prm.ws_lse + pl.n_part);
+  switch (G) {
+    case 1: launch_kernels<1>(prm, pl, stream); break;
+    case 2: launch_kernels<2>(prm, pl, stream); break;
+    case 4: launch_kernels<4>(prm, pl, stream); break;
+    default: launch_kernels<8>(prm, pl, stream); break;
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(FA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
   return FA_OK;
 }
 
@@ -329,53 +857,19 @@ int launch_decode(const void* q, const void* kcache, const void* vcache, const i
   const int G = Hq / Hkv;
   if (G != 1 && G != 2 && G != 4 && G != 8)
     return set_error(FA_ERR_UNSUPPORTED, "decode supports Hq/Hkv in {1,2,4,8} (got %d)", G);
-  DecodeParams prm;
-  prm.q = static_cast<const uint16_t*>(q);
-  prm.kc = static_cast<const uint16_t*>(kcache);
-  prm.vc = static_cast<const uint16_t*>(vcache);
-  prm.block_table = block_table;
-  prm.seq_lens = seq_lens;
-  prm.o = static_cast<uint16_t*>(o);
-  prm.lse = lse;
-  prm.B = B;
-  prm.Hq = Hq;
-  prm.Hkv = Hkv;
-  prm.max_pages = max_pages_per_seq;
-  prm.num_pages = num_pages;
-  // Pages per split: aim at ~2048 CTAs if every sequence were full length.
-  long long want = (static_cast<long long>(B) * max_pages_per_seq + 2047) / 2048;
-  int pps = 4;
-  while (pps < want && pps < 64) pps *= 2;
-  prm.pps = pps;
-  prm.nsplit = (max_pages_per_seq + pps - 1) / pps;
-  prm.scale_log2 = scale * kLog2e;
-  prm.err = device_error_word(device);
-  if (!prm.err) return set_error(FA_ERR_CUDA, "device error word unavailable");
-  if (prm.nsplit > 65535 || B > 65535)
-    return set_error(FA_ERR_UNSUPPORTED, "too many sequences or splits for one launch");
-
-  const size_t n_part = static_cast<size_t>(B) * prm.nsplit * Hq;
-  const size_t bytes = n_part * kDecD * sizeof(float) + n_part * sizeof(float);
+  const DecodePlan pl = make_plan(B, Hq, Hkv, max_pages_per_seq, sm_count(device));
   cudaMemPool_t pool;
   int rc = get_pool(device, &pool);
   if (rc != FA_OK) return rc;
   void* ws = nullptr;
-  cudaError_t e = cudaMallocFromPoolAsync(&ws, bytes, pool, stream);
+  cudaError_t e = cudaMallocFromPoolAsync(&ws, pl.bytes, pool, stream);
   if (e != cudaSuccess)
-    return set_error(FA_ERR_CUDA, "workspace allocation (%zu bytes): %s", bytes,
+    return set_error(FA_ERR_CUDA, "workspace allocation (%zu bytes): %s", pl.bytes,
                      cudaGetErrorString(e));
-  prm.ws_o = static_cast<float*>(ws);
-  prm.ws_lse = prm.ws_o + n_part * kDecD;
-  switch (G) {
-    case 1: launch_split<1>(prm, stream); break;
-    case 2: launch_split<2>(prm, stream); break;
-    case 4: launch_split<4>(prm, stream); break;
-    default: launch_split<8>(prm, stream); break;
-  }
-  fa_decode_combine_kernel<<<B * Hq, kDecD, 0, stream>>>(prm);
-  e = cudaGetLastError();
+  rc = run_decode(q, kcache, vcache, block_table, seq_lens, o, lse, B, Hq, Hkv, max_pages_per_seq,
+                  num_pages, scale, pl, ws, stream, device);
   cudaError_t ef = cudaFreeAsync(ws, stream);
-  if (e != cudaSuccess) return set_error(FA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+  if (rc != FA_OK) return rc;
   if (ef != cudaSuccess)
     return set_error(FA_ERR_CUDA, "workspace release: %s", cudaGetErrorString(ef));
   return FA_OK;
@@ -395,15 +889,15 @@ void release_decode_resources() {
 
 // ---------------------------------------------------------------- no-allocation variant
 //
-// Same split and combine kernels as launch_decode, but the chunk partials live
-// in a fixed array compiled into this library instead of memory obtained at
-// call time, for callers that cannot allocate device memory during a decode
-// step.  The array is part of the library's device image: every GPU on which
-// the library's kernels are loaded holds these bytes until the process exits.
-// Every call shares it and it keeps the previous call's contents; nothing in it
-// has to start at zero, because the merge only reads chunk results written
-// earlier in the same call.  Two calls whose kernels overlap on the GPU (for
-// example on two streams) use the same bytes and race.
+// Same kernels as launch_decode, but the chunk partials live in a fixed array
+// compiled into this library instead of memory obtained at call time, for
+// callers that cannot allocate device memory during a decode step.  The array
+// is part of the library's device image: every GPU on which the library's
+// kernels are loaded holds these bytes until the process exits.  Every call
+// shares it and it keeps the previous call's contents; nothing in it has to
+// start at zero when the call begins: each call writes everything it later reads
+// (the prefix offsets and every partial the merge reads).  Two calls whose kernels
+// overlap on the GPU (for example on two streams) use the same bytes and race.
 namespace fa {
 
 static __device__ __align__(256) float g_decode_scratch[kNoAllocScratchBytes / sizeof(float)];
@@ -429,79 +923,50 @@ int scratch_address(int device, float** out) {
   *out = g_scratch_ptr[device];
   return FA_OK;
 }
+
+// Plan that fits the fixed scratch: the streamed schedule as is when it fits;
+// the direct schedule with chunks widened until its partials fit.
+int plan_noalloc(int B, int Hq, int Hkv, int max_pages_per_seq, int nsm, DecodePlan* out) {
+  DecodePlan pl = make_plan(B, Hq, Hkv, max_pages_per_seq, nsm);
+  if (!pl.streamed) {
+    while (pl.bytes > kNoAllocScratchBytes && pl.nsplit > 1) {
+      pl.pps *= 2;
+      pl.nsplit = (max_pages_per_seq + pl.pps - 1) / pl.pps;
+      finish_plan(pl, B, Hq, Hkv);
+    }
+  }
+  if (pl.bytes > kNoAllocScratchBytes)
+    return set_error(FA_ERR_INVALID_ARG,
+                     "fa_decode_paged_noalloc: this problem needs %zu bytes of scratch; the fixed "
+                     "scratch holds %zu bytes (partial rows: (SMs + B) * Hq for Hkv <= 8, "
+                     "B * Hq for Hkv > 8, each %d bytes)",
+                     pl.bytes, kNoAllocScratchBytes, (kDecD + 1) * 4);
+  *out = pl;
+  return FA_OK;
+}
 }  // namespace
 
-int plan_decode_noalloc(int B, int Hq, int max_pages_per_seq, int* pps_out, int* nsplit_out) {
-  // Start from the split size launch_decode would use and widen the splits
-  // until the partials fit the fixed scratch array.
-  long long want = (static_cast<long long>(B) * max_pages_per_seq + 2047) / 2048;
-  long long pps = 4;
-  while (pps < want && pps < 64) pps *= 2;
-  for (;;) {
-    const long long nsplit = (max_pages_per_seq + pps - 1) / pps;
-    const long long bytes = static_cast<long long>(B) * nsplit * Hq * (kDecD + 1) * 4;
-    if (bytes <= static_cast<long long>(kNoAllocScratchBytes)) {
-      *pps_out = static_cast<int>(pps);
-      *nsplit_out = static_cast<int>(nsplit);
-      return FA_OK;
-    }
-    if (nsplit == 1)
-      return set_error(FA_ERR_INVALID_ARG,
-                       "fa_decode_paged_noalloc: B * Hq = %lld needs %lld bytes of scratch even "
-                       "with one chunk per sequence; the fixed scratch holds %zu bytes "
-                       "(B * Hq <= %zu)",
-                       static_cast<long long>(B) * Hq, bytes, kNoAllocScratchBytes,
-                       kNoAllocScratchBytes / ((kDecD + 1) * 4));
-    pps *= 2;
-  }
+int check_decode_noalloc(int B, int Hq, int Hkv, int max_pages_per_seq) {
+  // Host-side bound check (before the device is touched): the SM count is not
+  // known here, so the streamed schedule is checked against 148 SMs, the B200's.
+  DecodePlan pl;
+  return plan_noalloc(B, Hq, Hkv, max_pages_per_seq, 148, &pl);
 }
 
 int launch_decode_noalloc(const void* q, const void* kcache, const void* vcache,
                           const int32_t* block_table, const int32_t* seq_lens, void* o, float* lse,
                           int B, int Hq, int Hkv, int max_pages_per_seq, int num_pages,
                           float scale, cudaStream_t stream, int device) {
-  int pps = 0, nsplit = 0;
-  int rc = plan_decode_noalloc(B, Hq, max_pages_per_seq, &pps, &nsplit);
-  if (rc != FA_OK) return rc;
   const int G = Hq / Hkv;
   if (G != 1 && G != 2 && G != 4 && G != 8)
     return set_error(FA_ERR_UNSUPPORTED, "decode supports Hq/Hkv in {1,2,4,8} (got %d)", G);
+  DecodePlan pl;
+  int rc = plan_noalloc(B, Hq, Hkv, max_pages_per_seq, sm_count(device), &pl);
+  if (rc != FA_OK) return rc;
   float* scratch = nullptr;
   if ((rc = scratch_address(device, &scratch)) != FA_OK) return rc;
-  DecodeParams prm;
-  prm.q = static_cast<const uint16_t*>(q);
-  prm.kc = static_cast<const uint16_t*>(kcache);
-  prm.vc = static_cast<const uint16_t*>(vcache);
-  prm.block_table = block_table;
-  prm.seq_lens = seq_lens;
-  prm.o = static_cast<uint16_t*>(o);
-  prm.lse = lse;
-  prm.B = B;
-  prm.Hq = Hq;
-  prm.Hkv = Hkv;
-  prm.max_pages = max_pages_per_seq;
-  prm.num_pages = num_pages;
-  prm.pps = pps;
-  prm.nsplit = nsplit;
-  prm.scale_log2 = scale * kLog2e;
-  prm.err = device_error_word(device);
-  if (!prm.err) return set_error(FA_ERR_CUDA, "device error word unavailable");
-  if (nsplit > 65535 || B > 65535)
-    return set_error(FA_ERR_UNSUPPORTED, "too many sequences or splits for one launch");
-  const size_t n_part = static_cast<size_t>(B) * nsplit * Hq;
-  prm.ws_o = scratch;
-  prm.ws_lse = scratch + n_part * kDecD;
-  switch (G) {
-    case 1: launch_split<1>(prm, stream); break;
-    case 2: launch_split<2>(prm, stream); break;
-    case 4: launch_split<4>(prm, stream); break;
-    default: launch_split<8>(prm, stream); break;
-  }
-  fa_decode_combine_kernel<<<B * Hq, kDecD, 0, stream>>>(prm);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess)
-    return set_error(FA_ERR_CUDA, "decode (no-allocation) launch: %s", cudaGetErrorString(e));
-  return FA_OK;
+  return run_decode(q, kcache, vcache, block_table, seq_lens, o, lse, B, Hq, Hkv,
+                    max_pages_per_seq, num_pages, scale, pl, scratch, stream, device);
 }
 
 }  // namespace fa

@@ -8,11 +8,15 @@
 //
 // One CTA owns two 128-row query tiles (Q0, Q1) of one (batch, head) and streams
 // the 128-key K/V tiles of the matching KV head (GQA, devhandbook example 5)
-// through a ring of shared-memory slots.  Warp roles (320 threads):
-//   warps 0-3  softmax warpgroup for Q0   (thread r owns query row r = TMEM lane r)
-//   warps 4-7  softmax warpgroup for Q1
-//   warp  8    TMA producer: Q tiles once, then K_j, V_j into the slot ring
-//   warp  9    TMEM allocator and single-thread tcgen05 MMA issuer
+// through a ring of shared-memory slots.  Warp roles (384 threads, 3 warpgroups):
+//   warps 0-3   softmax warpgroup for Q0   (thread r owns query row r = TMEM lane r)
+//   warps 4-7   softmax warpgroup for Q1
+//   warp  8     TMA producer: Q tiles once, then K_j, V_j into the slot ring
+//   warp  9     TMEM allocator and single-thread tcgen05 MMA issuer
+//   warps 10-11 idle
+// The control warpgroup (warps 8-11) hands registers to the softmax warpgroups
+// (setmaxnreg): 72 and 216 per-thread registers over 128 + 256 threads equal
+// the 384 x 168 the block is launched with.
 // Tensor memory (512 columns x 128 lanes, fp32):
 //   [  0,128) S0 = Q0 K^T  (its first 64 columns are reused for P0 as bf16 pairs)
 //   [128,256) S1 = Q1 K^T  (P1 likewise)
@@ -21,7 +25,8 @@
 // tcgen05 operations of one thread execute in issue order, so S_{j+1} never
 // overwrites P_j before PV_j has read it, and the commit that publishes S_{j+1}
 // also guarantees PV_j finished -- the softmax warpgroup may then rescale O in
-// place before it releases P_{j+1}.
+// place before it releases P_{j+1}.  (The two query tiles' softmax phases
+// settle into alternation: each one's MMAs run while the other computes.)
 // The rescale is lazy: a row's reference maximum only moves when the new tile
 // maximum exceeds it by more than 2^8, so P stays <= 256 and O is rescaled only
 // on those rare tiles.  Exactness is unaffected: O and L share the reference.
@@ -39,7 +44,15 @@ namespace {
 constexpr int kBM = 128;       // query rows per tile = TMEM lanes
 constexpr int kBN = 128;       // keys per tile
 constexpr float kTau = 8.0f;   // lazy-rescale threshold (log2 units)
-constexpr int kThreads = 320;
+#ifndef FA_POLY_PAIRS
+#define FA_POLY_PAIRS 0
+#endif
+// Of every 16 column pairs, this many use the FMA-pipe exp2 (the rest use MUFU).
+constexpr int kPolyPairs = FA_POLY_PAIRS;
+constexpr int kThreads = 384;
+constexpr uint32_t kRegsControl = 72;    // warps 8-11
+constexpr uint32_t kRegsSoftmax = 216;   // warps 0-7
+static_assert(kRegsControl * 128 + kRegsSoftmax * 256 <= 384 * 168, "register split");
 
 template <int D>
 struct FwdLayout {
@@ -137,117 +150,127 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  if (warp == 8) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && n_max > 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      for (int t = 0; t < 2; ++t) {
-        if (n_kv[t] == 0) continue;
-        mbar_arrive_expect_tx(q_full(t), L::kTileBytes);
-        const uint32_t dst = sbase + L::kQOff + t * L::kTileBytes;
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_load_3d(dst + c * L::kChunkBytes, &tmQ, q_full(t), c * 64, q_row0 + t * kBM, bh);
-      }
-      const int kv_z = b * p.Hkv + hkv;
-      int issued = 0;
-      for (int j = 0; j < n_max; ++j) {
-        bool ok = true;
-        for (int w = 0; w < 2; ++w) {
-          const int pos = 2 * j + w;
-          const int slot = pos % L::kSlots;
-          const uint32_t ph = (pos / L::kSlots) & 1;
-          if (!mbar_wait(kv_empty(slot), ph ^ 1, abort_flag, p.err, p.timeout_ns)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(kv_full(slot), L::kTileBytes);
-          const uint32_t dst = sbase + L::kKVOff + slot * L::kTileBytes;
-          const void* tm = w ? static_cast<const void*>(&tmV) : static_cast<const void*>(&tmK);
+  if (warp >= 8) {
+    regs_dec<kRegsControl>();
+    if (warp == 8) {
+      // ------------------------------------------------------------ TMA producer
+      if (lane == 0 && n_max > 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        for (int t = 0; t < 2; ++t) {
+          if (n_kv[t] == 0) continue;
+          mbar_arrive_expect_tx(q_full(t), L::kTileBytes);
+          const uint32_t dst = sbase + L::kQOff + t * L::kTileBytes;
           for (int c = 0; c < L::kChunks; ++c)
-            tma_load_3d(dst + c * L::kChunkBytes, tm, kv_full(slot), c * 64, j * kBN, kv_z);
-          ++issued;
+            tma_load_3d(dst + c * L::kChunkBytes, &tmQ, q_full(t), c * 64, q_row0 + t * kBM, bh);
         }
-        if (!ok) break;
-      }
-      // Every issued copy must land before the CTA may exit (also on abort).
-      volatile int no_abort = 0;
-      for (int t = 0; t < 2; ++t)
-        if (n_kv[t] > 0) mbar_wait(q_full(t), 0, &no_abort, p.err, p.timeout_ns);
-      for (int s = 0; s < L::kSlots && s < issued; ++s) {
-        const int last = s + ((issued - 1 - s) / L::kSlots) * L::kSlots;
-        mbar_wait(kv_full(s), (last / L::kSlots) & 1, &no_abort, p.err, p.timeout_ns);
-      }
-    }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n_max > 0) {
-      constexpr uint32_t idesc_s = idesc_f16(kBM, kBN, BF16, false);
-      constexpr uint32_t idesc_pv = idesc_f16(kBM, D, BF16, true);
-      bool ok = true;
-      for (int t = 0; t < 2 && ok; ++t)
-        if (n_kv[t] > 0) ok = mbar_wait(q_full(t), 0, abort_flag, p.err, p.timeout_ns);
-      auto slot_of = [&](int pos) { return pos % L::kSlots; };
-      auto phase_of = [&](int pos) { return static_cast<uint32_t>((pos / L::kSlots) & 1); };
-      // S_t = Q_t K^T : M=128, N=128, K=D in steps of 16 (32 bytes inside a swizzle atom)
-      auto issue_s = [&](int t, int slot) {
-        const uint32_t qa = sbase + L::kQOff + t * L::kTileBytes;
-        const uint32_t kb = sbase + L::kKVOff + slot * L::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-          mma_ss(tmem + t * 128, smem_desc_sw128(qa + off, 16, 1024),
-                 smem_desc_sw128(kb + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(s_full(t));
-      };
-      // O_t += P_t V : A = P from TMEM (bf16 pairs), B = V tile, MN-major (D contiguous)
-      auto issue_pv = [&](int t, int slot, bool accumulate) {
-        const uint32_t vb = sbase + L::kKVOff + slot * L::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8,
-                 smem_desc_sw128(vb + kk * 16 * 128, L::kChunkBytes, 1024), idesc_pv,
-                 (accumulate || kk > 0) ? 1u : 0u);
-        }
-      };
-      if (ok) ok = mbar_wait(kv_full(slot_of(0)), phase_of(0), abort_flag, p.err, p.timeout_ns);
-      if (ok) {
-        tc_fence_after();
-        for (int t = 0; t < 2; ++t)
-          if (n_kv[t] > 0) issue_s(t, slot_of(0));
-        tc_commit(kv_empty(slot_of(0)));
-      }
-      for (int j = 0; j < n_max && ok; ++j) {
-        const int vpos = 2 * j + 1;
-        const int kpos = 2 * j + 2;
-        const bool has_next = j + 1 < n_max;
-        ok = mbar_wait(kv_full(slot_of(vpos)), phase_of(vpos), abort_flag, p.err, p.timeout_ns);
-        if (ok && has_next)
-          ok = mbar_wait(kv_full(slot_of(kpos)), phase_of(kpos), abort_flag, p.err, p.timeout_ns);
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (j >= n_kv[t]) continue;
-          ok = mbar_wait(p_full(t), j & 1, abort_flag, p.err, p.timeout_ns);
+        const int kv_z = b * p.Hkv + hkv;
+        int issued = 0;
+        for (int j = 0; j < n_max; ++j) {
+          bool ok = true;
+          for (int w = 0; w < 2; ++w) {
+            const int pos = 2 * j + w;
+            const int slot = pos % L::kSlots;
+            const uint32_t ph = (pos / L::kSlots) & 1;
+            if (!mbar_wait(kv_empty(slot), ph ^ 1, abort_flag, p.err, p.timeout_ns)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(kv_full(slot), L::kTileBytes);
+            const uint32_t dst = sbase + L::kKVOff + slot * L::kTileBytes;
+            const void* tm = w ? static_cast<const void*>(&tmV) : static_cast<const void*>(&tmK);
+            for (int c = 0; c < L::kChunks; ++c)
+              tma_load_3d(dst + c * L::kChunkBytes, tm, kv_full(slot), c * 64, j * kBN, kv_z);
+            ++issued;
+          }
           if (!ok) break;
-          tc_fence_after();
-          issue_pv(t, slot_of(vpos), j > 0);
-          if (j + 1 < n_kv[t])
-            issue_s(t, slot_of(kpos));
-          else
-            tc_commit(o_full(t));
         }
-        if (!ok) break;
-        tc_commit(kv_empty(slot_of(vpos)));
-        if (has_next) tc_commit(kv_empty(slot_of(kpos)));
+        // Every issued copy must land before the CTA may exit (also on abort).
+        volatile int no_abort = 0;
+        for (int t = 0; t < 2; ++t)
+          if (n_kv[t] > 0) mbar_wait(q_full(t), 0, &no_abort, p.err, p.timeout_ns);
+        for (int s = 0; s < L::kSlots && s < issued; ++s) {
+          const int last = s + ((issued - 1 - s) / L::kSlots) * L::kSlots;
+          mbar_wait(kv_full(s), (last / L::kSlots) & 1, &no_abort, p.err, p.timeout_ns);
+        }
       }
-      // All issued MMAs must complete before TMEM is released (also on abort).
-      tc_commit(mma_done);
-      volatile int no_abort = 0;
-      mbar_wait(mma_done, 0, &no_abort, p.err, p.timeout_ns);
-    }
+    } else if (warp == 9) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0 && n_max > 0) {
+        constexpr uint32_t idesc_s = idesc_f16(kBM, kBN, BF16, false);
+        constexpr uint32_t idesc_pv = idesc_f16(kBM, D, BF16, true);
+        auto slot_of = [&](int pos) { return pos % L::kSlots; };
+        auto phase_of = [&](int pos) { return static_cast<uint32_t>((pos / L::kSlots) & 1); };
+        // Descriptors are built once; moving to another K step or ring slot only
+        // adds (byte offset >> 4) to the start-address field in the low bits.
+        const uint64_t desc_q0 = smem_desc_sw128(sbase + L::kQOff, 16, 1024);
+        const uint64_t desc_q1 = smem_desc_sw128(sbase + L::kQOff + L::kTileBytes, 16, 1024);
+        const uint64_t desc_k = smem_desc_sw128(sbase + L::kKVOff, 16, 1024);            // K-major
+        const uint64_t desc_v = smem_desc_sw128(sbase + L::kKVOff, L::kChunkBytes, 1024);  // MN-major
+        // S_t = Q_t K^T : M=128, N=128, K=D in steps of 16 (32 bytes inside a swizzle atom)
+        auto issue_s = [&](int t, int slot) {
+          const uint64_t a0 = t ? desc_q1 : desc_q0;
+          const uint64_t b0 = desc_k + static_cast<uint64_t>((slot * L::kTileBytes) >> 4);
+          const uint32_t d = tmem + t * 128;
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * L::kChunkBytes + (kk & 3) * 32) >> 4);
+            mma_ss(d, a0 + off, b0 + off, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(s_full(t));
+        };
+        // O_t += P_t V : A = P from TMEM (bf16 pairs), B = V tile, MN-major (D contiguous)
+        auto issue_pv = [&](int t, int slot, bool accumulate) {
+          const uint64_t b0 = desc_v + static_cast<uint64_t>((slot * L::kTileBytes) >> 4);
+          const uint32_t d = tmem + 256 + t * D;
+          const uint32_t a = tmem + t * 128;
+  #pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            mma_ts(d, a + kk * 8, b0 + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_pv,
+                   (accumulate || kk > 0) ? 1u : 0u);
+        };
+        bool ok = true;
+        if (n_kv[0] > 0) ok = mbar_wait(q_full(0), 0, abort_flag, p.err, p.timeout_ns);
+        if (ok && n_kv[1] > 0) ok = mbar_wait(q_full(1), 0, abort_flag, p.err, p.timeout_ns);
+        if (ok) ok = mbar_wait(kv_full(slot_of(0)), phase_of(0), abort_flag, p.err, p.timeout_ns);
+        if (ok) {
+          tc_fence_after();
+          if (n_kv[0] > 0) issue_s(0, slot_of(0));
+          if (n_kv[1] > 0) issue_s(1, slot_of(0));
+          tc_commit(kv_empty(slot_of(0)));
+        }
+        for (int j = 0; j < n_max && ok; ++j) {
+          const int vpos = 2 * j + 1;
+          const int kpos = 2 * j + 2;
+          const bool has_next = j + 1 < n_max;
+          ok = mbar_wait(kv_full(slot_of(vpos)), phase_of(vpos), abort_flag, p.err, p.timeout_ns);
+          if (ok && has_next)
+            ok = mbar_wait(kv_full(slot_of(kpos)), phase_of(kpos), abort_flag, p.err, p.timeout_ns);
+  #pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (!ok || j >= (t ? n_kv[1] : n_kv[0])) continue;
+            ok = mbar_wait(p_full(t), j & 1, abort_flag, p.err, p.timeout_ns);
+            if (!ok) continue;
+            tc_fence_after();
+            issue_pv(t, slot_of(vpos), j > 0);
+            if (j + 1 < (t ? n_kv[1] : n_kv[0]))
+              issue_s(t, slot_of(kpos));
+            else
+              tc_commit(o_full(t));
+          }
+          if (!ok) break;
+          tc_commit(kv_empty(slot_of(vpos)));
+          if (has_next) tc_commit(kv_empty(slot_of(kpos)));
+        }
+        // All issued MMAs must complete before TMEM is released (also on abort).
+        tc_commit(mma_done);
+        volatile int no_abort = 0;
+        mbar_wait(mma_done, 0, &no_abort, p.err, p.timeout_ns);
+      }
+  }
   } else {
+    regs_inc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax warpgroups
     const int t = warp >> 2;
     const int r = tid & 127;
@@ -296,9 +319,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 128; ++e)
             if (e > lim) s[e] = __float_as_uint(-INFINITY);
         }
-        float mx = __uint_as_float(s[0]);
+        // row maximum: 8 independent three-input-max chains, then a short tree
+        float acc[8];
 #pragma unroll
-        for (int e = 1; e < 128; ++e) mx = fmaxf(mx, __uint_as_float(s[e]));
+        for (int k = 0; k < 8; ++k) acc[k] = __uint_as_float(s[k]);
+#pragma unroll
+        for (int e = 8; e + 16 <= 128; e += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            acc[k] = fmax3(acc[k], __uint_as_float(s[e + k]), __uint_as_float(s[e + 8 + k]));
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = fmaxf(acc[k], __uint_as_float(s[120 + k]));
+        const float mx = fmax3(fmax3(acc[0], acc[1], acc[2]), fmax3(acc[3], acc[4], acc[5]),
+                               fmaxf(acc[6], acc[7]));
         const float m_tile = mx * p.scale_log2;
         const bool move = m_tile > m_used + kTau;
         float alpha = 1.f;
@@ -321,21 +354,51 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
-        float sum = 0.f;
+        const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t nm2 = f2_pack(neg_m, neg_m);
+        uint64_t sum2[4] = {0, 0, 0, 0};   // four independent packed partial sums
+        if (need_mask) {
+          // masked tiles: every exponential on MUFU (exactly 0 for masked scores)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float p0 = ex2(fmaf(__uint_as_float(s[32 * c + 2 * e]), p.scale_log2, neg_m));
-            const float p1 =
-                ex2(fmaf(__uint_as_float(s[32 * c + 2 * e + 1]), p.scale_log2, neg_m));
-            sum += p0 + p1;
-            pk[e] = BF16 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
+            for (int e = 0; e < 16; ++e) {
+              float x0, x1;
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(s[32 * c + 2 * e]),
+                                       __uint_as_float(s[32 * c + 2 * e + 1])), c2, nm2), x0, x1);
+              const float p0 = ex2(x0), p1 = ex2(x1);
+              sum2[e & 3] = f2_add(sum2[e & 3], f2_pack(p0, p1));
+              pk[e] = BF16 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
+            }
+            tmem_st16(tS + 16 * c, pk);
           }
-          tmem_st16(tS + 16 * c, pk);
+        } else {
+          // unmasked tiles: the first kPolyPairs pairs of every 32 columns on the
+          // FMA pipe, the rest on MUFU, so both units share the exponentials
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              float x0, x1, p0, p1;
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(s[32 * c + 2 * e]),
+                                       __uint_as_float(s[32 * c + 2 * e + 1])), c2, nm2), x0, x1);
+              if (e < kPolyPairs) {
+                exp2_fma_pair(x0, x1, p0, p1);
+              } else {
+                p0 = ex2(x0);
+                p1 = ex2(x1);
+              }
+              sum2[e & 3] = f2_add(sum2[e & 3], f2_pack(p0, p1));
+              pk[e] = BF16 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
+            }
+            tmem_st16(tS + 16 * c, pk);
+          }
         }
-        l += sum;
+        float sa, sb;
+        f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), sa, sb);
+        l += sa + sb;
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(p_full(t));

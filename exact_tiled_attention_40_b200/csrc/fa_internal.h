@@ -34,9 +34,9 @@ void release_decode_resources();
 // Size of the fixed scratch array used by fa_decode_paged_noalloc.
 constexpr size_t kNoAllocScratchBytes = 16u << 20;   // 16 MiB
 
-// Chunking for fa_decode_paged_noalloc: pages per split and split count such
-// that the partials fit kNoAllocScratchBytes (host only; no device needed).
-int plan_decode_noalloc(int B, int Hq, int max_pages_per_seq, int* pps, int* nsplit);
+// Host-side check that a problem fits the fixed scratch of
+// fa_decode_paged_noalloc (no device needed).  Returns an FA_* status.
+int check_decode_noalloc(int B, int Hq, int Hkv, int max_pages_per_seq);
 
 // Split-KV paged decode whose partials live in the library's fixed scratch
 // array; allocates nothing.  `device` must be the current device.

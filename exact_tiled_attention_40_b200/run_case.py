@@ -1,0 +1,74 @@
+"""Run one named workload through the library and print per-launch times.
+
+    python -m exact_tiled_attention_40_b200.run_case --case gqa_b1_hq32_hkv8_n8192_d128_causal
+    python -m exact_tiled_attention_40_b200.run_case --case decode_b64_hq32_hkv8_d128_page16
+
+Inputs come from the seeded generator and stay resident on the device; a
+256 MiB buffer is written before every launch so no launch finds its inputs in
+L2.  Each launch is timed with CUDA events on the launching stream.  Handy for
+profiling one kernel on one workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import statistics
+
+import torch
+
+from . import fa
+from .inputs import DECODE_CASES, PREFILL_CASES, make_decode, make_prefill
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--case", required=True,
+                    choices=sorted(PREFILL_CASES) + sorted(DECODE_CASES))
+    ap.add_argument("--iters", type=int, default=5)
+    args = ap.parse_args()
+    dev = torch.device("cuda", 0)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    if args.case in PREFILL_CASES:
+        c = PREFILL_CASES[args.case]
+        q, k, v, _ = make_prefill(c)
+        q, k, v = q.to(dev), k.to(dev), v.to(dev)
+        o = torch.empty_like(q)
+        lse = torch.empty((c.B, c.Hq, c.Nq), dtype=torch.float32, device=dev)
+
+        def launch():
+            fa.fa_fwd(q, k, v, o, lse, c.B, c.Hq, c.Hkv, c.Nq, c.Nk, c.D, c.softmax_scale,
+                      c.causal, stream=stream.cuda_stream)
+        work, unit = c.flops / 1e12, "TFLOP/s"
+    else:
+        c = DECODE_CASES[args.case]
+        q, kc, vc, table, lens = make_decode(c)
+        q, kc, vc, table, lens = (t.to(dev) for t in (q, kc, vc, table, lens))
+        o = torch.empty_like(q)
+        lse = torch.empty((c.B, c.Hq), dtype=torch.float32, device=dev)
+
+        def launch():
+            fa.fa_decode_paged(q, kc, vc, table, lens, o, c.B, c.Hq, c.Hkv, c.D, c.page_size,
+                               c.softmax_scale, table.shape[1], c.num_pages, lse,
+                               stream=stream.cuda_stream)
+        work, unit = int(lens.sum()) * c.Hkv * c.D * 2 * 2 / 1e9, "GB/s"
+    times = []
+    for i in range(args.iters):
+        flush.fill_(i & 0xff)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        launch()
+        b.record(stream)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    if fa.device_status() != 0:
+        raise SystemExit(fa.last_error())
+    best = min(times)
+    print(json.dumps({"case": args.case, "ms": times, "best_ms": best,
+                      "median_ms": statistics.median(times),
+                      "rate_at_median": work / (statistics.median(times) * 1e-3), "unit": unit}))
+
+
+if __name__ == "__main__":
+    main()

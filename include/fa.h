@@ -88,14 +88,16 @@ int fa_fwd_fp16(const void* q, const void* k, const void* v, void* o, float* lse
  *   seq_lens    [B] int32, 0 <= seq_lens[b] <= max_pages_per_seq * page_size
  *   o           [B, Hq, D] bf16 (written)
  *   lse         [B, Hq] fp32 (written; may be NULL)
- * Supported: D == 128, page_size == 16, Hq / Hkv in {1, 2, 4, 8, 16}.
+ * Supported: D == 128, page_size == 16, Hq / Hkv in {1, 2, 4, 8}.
  * num_pages bounds every block-table entry (0 <= id < num_pages); entries out
  * of range are skipped and flagged in the device error word.
  * A sequence of length 0 gets O = 0 and LSE = -inf.
  * Work is split over key chunks; partial results are merged by their LSE.
- * The partials live in a stream-ordered workspace taken from a library-owned
- * memory pool on `stream` and returned to it on `stream` (no device sync);
- * fa_release() frees the pool.
+ * For Hkv <= 8 and Hq/Hkv <= 4 one persistent CTA per SM takes an equal share of all
+ * sequences' cache (so ragged lengths stay balanced); otherwise the grid is
+ * (chunk, sequence).  The partials live in a stream-ordered workspace taken
+ * from a library-owned memory pool on `stream` and returned to it on `stream`
+ * (no device sync); fa_release() frees the pool.
  */
 int fa_decode_paged(const void* q, const void* kcache, const void* vcache,
                     const int32_t* block_table, const int32_t* seq_lens, void* o, int B, int Hq,
@@ -117,11 +119,13 @@ int fa_decode_paged(const void* q, const void* kcache, const void* vcache,
  *
  * Arguments, layouts, supported sizes, outputs and error codes are those of
  * fa_decode_paged.  Differences:
- *   - The chunking is widened until the partials fit the array; the result
- *     agrees with fa_decode_paged within rounding, not bit for bit.
- *   - Problems whose partials do not fit even with one chunk per sequence
- *     (B * Hq > 32,513 at D = 128) are rejected with FA_ERR_INVALID_ARG before
- *     anything touches the device.
+ *   - The partial results need (number of SMs + B) * Hq rows of 516 bytes when
+ *     Hkv <= 8 and Hq/Hkv <= 4 (on a 148-SM B200: (148 + B) * Hq <= 32,513), and
+ *     B * Hq * chunks
+ *     rows otherwise, the chunks being widened until they fit (then the result
+ *     agrees with fa_decode_paged within rounding, not bit for bit).  Larger
+ *     problems are rejected with FA_ERR_INVALID_ARG before anything touches the
+ *     device.
  *   - The array is shared by every call and keeps the previous call's contents
  *     (nothing in it needs to start at zero).  Calls whose kernels overlap on
  *     the GPU, e.g. issued on two streams without ordering, race on it.

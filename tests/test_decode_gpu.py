@@ -37,7 +37,7 @@ def check(case, q, kc, vc, table, lens):
     assert np.all(lse.numpy()[~live] == -np.inf)
 
 
-@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (4, 4), (8, 4), (16, 2)])
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (4, 4), (8, 4), (16, 2), (32, 16)])
 def test_small_decode_matches_oracle(cuda_device, Hq, Hkv):
     case = DecodeCase("small", 5, Hq, Hkv, 128, 16, 1, 700, 300, seed=40 + Hq + Hkv)
     q, kc, vc, table, lens = make_decode(case)
@@ -45,6 +45,13 @@ def test_small_decode_matches_oracle(cuda_device, Hq, Hkv):
     lens[1] = 16       # exactly one page
     lens[2] = 17       # one page plus one token
     check(case, q, kc, vc, table, lens)
+
+
+def test_fewer_cache_chunks_than_sms(cuda_device):
+    """Short sequences: far fewer 8-token chunks than SMs, so most persistent
+    CTAs get an empty share and the merge must skip them."""
+    case = DecodeCase("short", 6, 16, 4, 128, 16, 1, 20, 40, seed=52)
+    check(case, *make_decode(case))
 
 
 def test_zero_length_sequence(cuda_device):

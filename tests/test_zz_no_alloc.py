@@ -22,8 +22,7 @@ FAKE = 0x10000
 
 def test_oversized_problem_is_rejected_before_touching_the_device():
     lib = fa.lib()
-    # B * Hq = 40000 > 32513: the partials cannot fit the fixed scratch even
-    # with one chunk per sequence.
+    # (148 + B) * Hq = 44,736 > 32,513 rows: the partials cannot fit the fixed scratch.
     rc = lib.fa_decode_paged_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1250, 32, 8, 128, 16,
                                      0.1, None, 4, 100, None)
     assert rc == 1                                         # FA_ERR_INVALID_ARG
