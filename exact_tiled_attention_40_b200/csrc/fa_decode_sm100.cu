@@ -19,19 +19,20 @@
 // Attention", formula 2.
 //
 // Two schedules:
-//  * Hkv <= 8 and Hq/Hkv <= 4 (streamed): one persistent CTA per SM.  All sequences' caches form
+//  * Hkv <= 8 (streamed): one persistent CTA per SM.  All sequences' caches form
 //    one list of half-pages (8 token slots: 8 * Hkv * 256 bytes of K and as many
 //    of V, each contiguous in the pool); CTA c takes the equal share
 //    [c*H/C, (c+1)*H/C) of the H half-pages, whatever the sequence lengths.  A
-//    producer warp streams them through a shared-memory ring with bulk async
-//    copies; eight consumer warps (warp g <-> KV head g; 8 lanes per token,
-//    4 tokens per instruction) compute from shared memory and emit one partial
-//    result per (CTA, sequence) segment, stored in
+//    producer warp streams them through a shared-memory ring with TMA tensor
+//    copies (128-byte swizzle, head-major boxes); eight consumer warps (warp g <-> KV head g) compute scores and
+//    outputs with warp-level tensor-core MMAs from shared memory and emit one
+//    partial result per (CTA, sequence) segment, stored in
 //    slot c + b (unique: along the list either c or b or both grow by one); a
 //    merge kernel combines each sequence's segments.
 //  * otherwise (direct): grid (chunk, sequence) of fixed page chunks, cache read
 //    straight from HBM with 16-byte non-allocating loads.
 #include <cstdio>
+#include <cstring>
 #include <mutex>
 #include <vector>
 
@@ -123,29 +124,6 @@ __device__ __forceinline__ float fold_heads(float (&v)[G], int sub) {
   float x = v[0];
 #pragma unroll
   for (int mask = 8 >> LG; mask >= 1; mask >>= 1) x += __shfl_xor_sync(0xffffffffu, x, mask);
-  return x;
-}
-
-// Same fold over the 8 slice lanes of a token (lane bits 0-2 = ls): lane `ls`
-// ends with the total of head ls >> (3 - log2 G).
-template <int G>
-__device__ __forceinline__ float fold_heads8(float (&v)[G], int ls) {
-  constexpr int LG = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3;
-#pragma unroll
-  for (int step = 0; step < LG; ++step) {
-    const int mask = 4 >> step;
-    const bool upper = (ls & mask) != 0;
-    const int n = G >> (step + 1);
-#pragma unroll
-    for (int k = 0; k < n; ++k) {
-      const float keep = upper ? v[k + n] : v[k];
-      const float send = upper ? v[k] : v[k + n];
-      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
-    }
-  }
-  float x = v[0];
-#pragma unroll
-  for (int mask = 4 >> LG; mask >= 1; mask >>= 1) x += __shfl_xor_sync(0xffffffffu, x, mask);
   return x;
 }
 
@@ -302,7 +280,12 @@ __global__ void __launch_bounds__(kDecThreads) fa_decode_split_kernel(const Deco
 }
 
 
-__host__ __device__ constexpr int half_bytes(int Hkv) { return kHalf * Hkv * kDecD * 2; }
+// A stage holds, for K and for V, two TMA boxes (head dimension halves) of
+// [Hkv heads][8 tokens][64 elements] with 128-byte swizzle: the 128-byte row of
+// (head g, token t) keeps its 16-byte chunk c at position c ^ t, so the 8 token
+// rows of one head are read by ldmatrix without bank conflicts.
+__host__ __device__ constexpr int box_bytes(int Hkv) { return Hkv * kHalf * 64 * 2; }
+__host__ __device__ constexpr int stage_kv_bytes(int Hkv) { return 2 * box_bytes(Hkv); }
 
 // hb[b] = sum over b' < b of ceil(len_b' / 8); hb[B] = total.  One block.
 __global__ void __launch_bounds__(1024) fa_decode_scan_kernel(const DecodeParams p) {
@@ -362,14 +345,15 @@ struct StageMeta {
 };
 
 template <int G>
-__global__ void __launch_bounds__(kStreamThreads, 1) fa_decode_stream_kernel(const DecodeParams p) {
-  // Consumer warp g owns KV head g and all G query heads that share it, so
-  // every K/V byte is read once from shared memory.
-  constexpr int GW = G;                          // query heads per warp
-  constexpr int LG = GW == 1 ? 0 : GW == 2 ? 1 : GW == 4 ? 2 : 3;
-  constexpr int SHIFT = 3 - LG;                  // slice lane `h << SHIFT` holds head h after the fold
-  constexpr int NQ = kHalf / 4;                  // token quads per stage
-  extern __shared__ __align__(128) uint8_t dsm[];
+__global__ void __launch_bounds__(kStreamThreads, 1)
+    fa_decode_stream_kernel(const __grid_constant__ CUtensorMap tmK,
+                            const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
+  // Consumer warp g owns KV head g and its G <= 8 query heads.  Scores and
+  // outputs use warp-level tensor-core MMAs: S (16 x 8) = Q (16 query-head rows,
+  // G used) x K^T per 8-token stage, then O (16 x 128) += P (16 x 8) x V; the
+  // score fragment becomes the P operand in registers, and every lane's rows
+  // are its own query head, so the online softmax needs no broadcasts.
+  extern __shared__ __align__(1024) uint8_t dsm_raw[];
   __shared__ __align__(8) uint64_t bars[2 * kMaxStages];
   __shared__ StageMeta meta[kMaxStages];
   __shared__ int abort_sm;
@@ -385,8 +369,10 @@ __global__ void __launch_bounds__(kStreamThreads, 1) fa_decode_stream_kernel(con
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int NS = p.nstages;
-  const int SB = half_bytes(p.Hkv);
-  const uint32_t sbase = smem_u32(dsm);
+  const int HB = box_bytes(p.Hkv);              // one TMA box (half of the head dimension)
+  const int SKV = stage_kv_bytes(p.Hkv);        // bytes per stage for K (and for V)
+  // swizzled TMA destinations must be 1024-byte aligned
+  const uint32_t sbase = (smem_u32(dsm_raw) + 1023u) & ~1023u;
   auto full = [&](int st) { return smem_u32(&bars[st]); };
   auto empty = [&](int st) { return smem_u32(&bars[kMaxStages + st]); };
   volatile int* abort_flag = &abort_sm;
@@ -447,10 +433,13 @@ __global__ void __launch_bounds__(kStreamThreads, 1) fa_decode_stream_kernel(con
             md.flags = kflags;
             meta[st] = md;
             if (kflags & 4) {
-              const size_t tok0 = static_cast<size_t>(kpage) * kPage + (khh & 1) * kHalf;
-              mbar_arrive_expect_tx(full(st), 2 * SB);
-              bulk_load(sbase + st * 2 * SB, p.kc + tok0 * p.Hkv * kDecD, SB, full(st));
-              bulk_load(sbase + st * 2 * SB + SB, p.vc + tok0 * p.Hkv * kDecD, SB, full(st));
+              const int tok0 = kpage * kPage + (khh & 1) * kHalf;
+              const uint32_t kdst = sbase + st * 2 * SKV;
+              mbar_arrive_expect_tx(full(st), 2 * SKV);
+              tma_load_3d(kdst, &tmK, full(st), 0, tok0, 0);
+              tma_load_3d(kdst + HB, &tmK, full(st), 64, tok0, 0);
+              tma_load_3d(kdst + SKV, &tmV, full(st), 0, tok0, 0);
+              tma_load_3d(kdst + SKV + HB, &tmV, full(st), 64, tok0, 0);
             } else {
               atomicOr(p.err, kErrBadIndex);   // consumers skip this stage
               mbar_arrive(full(st));
@@ -473,145 +462,103 @@ __global__ void __launch_bounds__(kStreamThreads, 1) fa_decode_stream_kernel(con
 
   regs_inc<kRegsConsumer>();
   // ------------------------------------------------------------------ consumers
-  // Lane = 8 * tq + ls: the warp takes 4 tokens at a time (tq), and each token's
-  // 256-byte head row is split over 8 lanes of 32 bytes (16 elements, ls).
-  const int tq = lane >> 3;
-  const int ls = lane & 7;
-  const int my_head = ls >> SHIFT;
+  // Fragment layout (m16n8k16 / m16n8k8, gq = lane / 4, tq = lane % 4): score and
+  // output rows are query heads gq (rows gq + 8 are unused and stay zero),
+  // columns are tokens 2 tq, 2 tq + 1 of the stage (scores) or output columns
+  // 8 n + 2 tq, 8 n + 2 tq + 1 (chunk n of O).
+  const int gq = lane >> 2;
+  const int tq = lane & 3;
   const int g = warp;                          // KV head of this warp (idle when g >= Hkv)
   const bool active = g < p.Hkv;
-  const int hq0 = g * G;
-  const int row_bytes = p.Hkv * kDecD * 2;
-  uint64_t q2[GW][8];
-  uint64_t acc2[GW][8];
-  float m[GW], l[GW];
-  float m_mine = -INFINITY;
+  const bool my_row = gq < G;                  // this lane's rows are real query heads
+  const int hq = g * G + (my_row ? gq : 0);
+  uint32_t qa[8][2];                           // Q A-fragments per 16-wide d chunk
+  float o[16][4];
+  float m_run = -INFINITY, l_run = 0.f;
+  // ldmatrix: lane supplies row (head g, token lane % 8) of matrix lane / 8; for the
+  // 32-wide group dg that is swizzled chunk ((dg & 1) * 4 + lane / 8) ^ (lane % 8)
+  // in box dg / 2.
+  const int lt = lane & 7;
+  const uint32_t row_off = static_cast<uint32_t>((g * kHalf + lt) * 128);
+  uint32_t ld_off[4];
+#pragma unroll
+  for (int dg = 0; dg < 4; ++dg)
+    ld_off[dg] = static_cast<uint32_t>((dg >> 1) * HB) + row_off +
+                 static_cast<uint32_t>((((dg & 1) * 4 + (lane >> 3)) ^ lt) << 4);
   for (int i = 0; i < n; ++i) {
     const int st = i % NS;
-    const bool got = mbar_wait(full(st), (i / NS) & 1, abort_flag, p.err, kWaitLimitNs);
-    if (!__all_sync(0xffffffffu, got)) return;
+    const bool ready = mbar_wait(full(st), (i / NS) & 1, abort_flag, p.err, kWaitLimitNs);
+    if (!__all_sync(0xffffffffu, ready)) return;
     const StageMeta md = meta[st];
     if (active) {
       if (md.flags & 1) {                      // a new sequence segment begins
-        m_mine = -INFINITY;
+        m_run = -INFINITY;
+        l_run = 0.f;
+        const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+            p.q + (static_cast<size_t>(md.b) * p.Hq + hq) * kDecD);
 #pragma unroll
-        for (int h = 0; h < GW; ++h) {
-          m[h] = -INFINITY;
-          l[h] = 0.f;
-          const uint4* qp = reinterpret_cast<const uint4*>(
-              p.q + (static_cast<size_t>(md.b) * p.Hq + hq0 + h) * kDecD + ls * 16);
-#pragma unroll
-          for (int v = 0; v < 2; ++v) {
-            const uint4 u = qp[v];
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              acc2[h][4 * v + e] = 0;
-              q2[h][4 * v + e] = f2_pack(__uint_as_float(w[e] << 16) * p.scale_log2,
-                                         __uint_as_float(w[e] & 0xffff0000u) * p.scale_log2);
-            }
-          }
+        for (int kc = 0; kc < 8; ++kc) {
+          qa[kc][0] = my_row ? qrow[kc * 8 + tq] : 0u;       // elements 16 kc + 2 tq, +1
+          qa[kc][1] = my_row ? qrow[kc * 8 + 4 + tq] : 0u;   // elements 16 kc + 8 + 2 tq, +1
         }
+#pragma unroll
+        for (int nn = 0; nn < 16; ++nn) o[nn][0] = o[nn][1] = o[nn][2] = o[nn][3] = 0.f;
       }
       if (md.flags & 4) {
         const int ntok = min(kHalf, md.len - md.hh * kHalf);
-        const uint8_t* kst = dsm + st * 2 * SB + (g * kDecD + ls * 16) * 2;
-        const uint8_t* vst = kst + SB;
-        float sc[NQ];
+        const uint32_t kaddr = sbase + st * 2 * SKV;
+        const uint32_t vaddr = kaddr + SKV;
+        // S = Q K^T over the 128-wide head dimension, 32 columns per ldmatrix
+        float sa[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int qd = 0; qd < NQ; ++qd) {
-          const int t = 4 * qd + tq;
-          const uint4* kp = reinterpret_cast<const uint4*>(kst + t * row_bytes);
-          const uint4 k0 = kp[0], k1 = kp[1];
-          const uint32_t w[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-          float partial[GW];
-#pragma unroll
-          for (int h = 0; h < GW; ++h) {
-            uint64_t a2 = 0;
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              a2 = f2_fma(q2[h][e], f2_pack(__uint_as_float(w[e] << 16),
-                                            __uint_as_float(w[e] & 0xffff0000u)), a2);
-            float lo2, hi2;
-            f2_unpack(a2, lo2, hi2);
-            partial[h] = lo2 + hi2;
-          }
-          sc[qd] = fold_heads8<GW>(partial, ls);
-          if (t >= ntok) sc[qd] = -INFINITY;
+        for (int dg = 0; dg < 4; ++dg) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(kaddr + ld_off[dg], b0, b1, b2, b3);
+          mma_bf16_16816(sa, qa[2 * dg][0], 0u, qa[2 * dg][1], 0u, b0, b1);
+          mma_bf16_16816(sa, qa[2 * dg + 1][0], 0u, qa[2 * dg + 1][1], 0u, b2, b3);
         }
-        // stage maximum of this lane's head over its tokens and the other 3 token lanes
-        float mx = sc[0];
+        const int t0 = 2 * tq;
+        const float s0 = t0 < ntok ? sa[0] * p.scale_log2 : -INFINITY;
+        const float s1 = t0 + 1 < ntok ? sa[1] * p.scale_log2 : -INFINITY;
+        float mx = fmaxf(s0, s1);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const float m_new = fmaxf(m_run, mx);
+        const float alpha = (m_run == -INFINITY) ? 0.f : ex2(m_run - m_new);
+        m_run = m_new;
+        const float p0 = (s0 == -INFINITY) ? 0.f : ex2(s0 - m_run);
+        const float p1 = (s1 == -INFINITY) ? 0.f : ex2(s1 - m_run);
+        l_run = l_run * alpha + (p0 + p1);
+        const uint32_t pa = pack_bf16x2(p0, p1);   // P A-fragment: row gq, tokens 2 tq, 2 tq + 1
 #pragma unroll
-        for (int qd = 1; qd < NQ; ++qd) mx = fmaxf(mx, sc[qd]);
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        m_mine = fmaxf(m_mine, mx);
-#pragma unroll
-        for (int h = 0; h < GW; ++h) {
-          const float mh = fmaxf(m[h], __shfl_sync(0xffffffffu, mx, h << SHIFT));
-          const float alpha = (m[h] == -INFINITY) ? 0.f : ex2(m[h] - mh);
-          l[h] *= alpha;
-          const uint64_t a2 = f2_pack(alpha, alpha);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc2[h][e] = f2_mul(acc2[h][e], a2);
-          m[h] = mh;
+        for (int nn = 0; nn < 16; ++nn) {
+          o[nn][0] *= alpha;
+          o[nn][1] *= alpha;
         }
-        float pv[NQ];
-        float psum = 0.f;
 #pragma unroll
-        for (int qd = 0; qd < NQ; ++qd) {
-          pv[qd] = (sc[qd] == -INFINITY) ? 0.f : ex2(sc[qd] - m_mine);
-          psum += pv[qd];
-        }
-        psum += __shfl_xor_sync(0xffffffffu, psum, 8);
-        psum += __shfl_xor_sync(0xffffffffu, psum, 16);
-#pragma unroll
-        for (int h = 0; h < GW; ++h) l[h] += __shfl_sync(0xffffffffu, psum, h << SHIFT);
-#pragma unroll
-        for (int qd = 0; qd < NQ; ++qd) {
-          const int t = 4 * qd + tq;
-          // slots past the sequence end hold arbitrary bytes: their V must not
-          // meet a zero weight as NaN * 0
-          uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
-          if (t < ntok) {
-            const uint4* vp = reinterpret_cast<const uint4*>(vst + t * row_bytes);
-            v0 = vp[0];
-            v1 = vp[1];
-          }
-          const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-          for (int h = 0; h < GW; ++h) {
-            // weight of (token t, head h) from the lane of the same token holding head h
-            const float pp = __shfl_sync(0xffffffffu, pv[qd], (tq << 3) | (h << SHIFT));
-            const uint64_t p2 = f2_pack(pp, pp);
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              acc2[h][e] = f2_fma(p2, f2_pack(__uint_as_float(w[e] << 16),
-                                              __uint_as_float(w[e] & 0xffff0000u)), acc2[h][e]);
-          }
+        for (int ng = 0; ng < 4; ++ng) {
+          uint32_t v0, v1, v2, v3;
+          ldsm_x4_t(vaddr + ld_off[ng], v0, v1, v2, v3);
+          mma_bf16_1688(o[4 * ng + 0], pa, 0u, v0);
+          mma_bf16_1688(o[4 * ng + 1], pa, 0u, v1);
+          mma_bf16_1688(o[4 * ng + 2], pa, 0u, v2);
+          mma_bf16_1688(o[4 * ng + 3], pa, 0u, v3);
         }
       }
+
       if (md.flags & 2) {                      // segment ends: write its partial to slot c + b
-        const size_t base = (static_cast<size_t>(c) + md.b) * p.Hq + hq0;
+        float l_tot = l_run;
+        l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 1);
+        l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 2);
+        if (my_row) {
+          const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
+          const size_t rowi = (static_cast<size_t>(c) + md.b) * p.Hq + hq;
+          float* dst = p.ws_o + rowi * kDecD + 2 * tq;
 #pragma unroll
-        for (int h = 0; h < GW; ++h) {
-          const float inv = l[h] > 0.f ? 1.f / l[h] : 0.f;
-          float4* dst = reinterpret_cast<float4*>(p.ws_o + (base + h) * kDecD + ls * 16);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            float a4[4];
-            f2_unpack(acc2[h][2 * v], a4[0], a4[1]);
-            f2_unpack(acc2[h][2 * v + 1], a4[2], a4[3]);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              // the four token lanes accumulated different tokens of the same slice
-              a4[e] += __shfl_xor_sync(0xffffffffu, a4[e], 8);
-              a4[e] += __shfl_xor_sync(0xffffffffu, a4[e], 16);
-            }
-            if (tq == 0) dst[v] = make_float4(a4[0] * inv, a4[1] * inv, a4[2] * inv, a4[3] * inv);
-          }
-          if (tq == 0 && ls == 0)
-            p.ws_lse[base + h] = l[h] > 0.f ? (m[h] + __log2f(l[h])) * kLn2 : -INFINITY;
+          for (int nn = 0; nn < 16; ++nn)
+            *reinterpret_cast<float2*>(dst + 8 * nn) = make_float2(o[nn][0] * inv, o[nn][1] * inv);
+          if (tq == 0)
+            p.ws_lse[rowi] = l_tot > 0.f ? (m_run + __log2f(l_tot)) * kLn2 : -INFINITY;
         }
       }
     }
@@ -766,11 +713,11 @@ void finish_plan(DecodePlan& pl, int B, int Hq, int Hkv) {
 
 DecodePlan make_plan(int B, int Hq, int Hkv, int max_pages_per_seq, int nsm) {
   DecodePlan pl;
-  // streamed: one consumer warp per KV head holds the state of G <= 4 query heads
-  pl.streamed = Hkv <= kDecWarps && Hq / Hkv <= 4 && nsm > 0;
+  // streamed: one consumer warp per KV head, its G <= 8 query heads as MMA rows
+  pl.streamed = Hkv <= kDecWarps && nsm > 0;
   if (pl.streamed) {
     pl.nctas = nsm;
-    pl.nstages = kStreamSmemBudget / (2 * half_bytes(Hkv));
+    pl.nstages = kStreamSmemBudget / (2 * stage_kv_bytes(Hkv));
     if (pl.nstages > kMaxStages) pl.nstages = kMaxStages;
   } else {
     pl.pps = direct_pps(B, max_pages_per_seq);
@@ -781,18 +728,18 @@ DecodePlan make_plan(int B, int Hq, int Hkv, int max_pages_per_seq, int nsm) {
 }
 
 template <int G>
-void launch_kernels(const DecodeParams& prm, const DecodePlan& pl, cudaStream_t stream) {
-  if (G <= 4 && pl.streamed) {
-    const int smem = pl.nstages * 2 * half_bytes(prm.Hkv);
+void launch_kernels(const DecodeParams& prm, const DecodePlan& pl, const CUtensorMap& tmK,
+                    const CUtensorMap& tmV, cudaStream_t stream) {
+  if (pl.streamed) {
+    const int smem = pl.nstages * 2 * stage_kv_bytes(prm.Hkv) + 1024;
     static bool attr_done = false;   // the attribute belongs to the function, per process
     if (!attr_done) {
-      cudaFuncSetAttribute(fa_decode_stream_kernel<(G <= 4 ? G : 4)>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kStreamSmemBudget);
+      cudaFuncSetAttribute(fa_decode_stream_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kStreamSmemBudget + 1024);
       attr_done = true;
     }
     fa_decode_scan_kernel<<<1, 1024, 0, stream>>>(prm);
-    fa_decode_stream_kernel<(G <= 4 ? G : 4)><<<pl.nctas, kStreamThreads, smem, stream>>>(prm);
+    fa_decode_stream_kernel<G><<<pl.nctas, kStreamThreads, smem, stream>>>(tmK, tmV, prm);
     fa_decode_stream_merge_kernel<<<(prm.B * prm.Hq + 3) / 4, 128, 0, stream>>>(prm);
   } else {
     dim3 grid(pl.nsplit, prm.B);
@@ -834,11 +781,27 @@ int run_decode(const void* q, const void* kcache, const void* vcache, const int3
   prm.ws_o = static_cast<float*>(ws);
   prm.ws_lse = prm.ws_o + pl.n_part * kDecD;
   prm.hb = reinterpret_cast<int*>(prm.ws_lse + pl.n_part);
+  CUtensorMap tmK, tmV;
+  if (pl.streamed) {
+    // K and V caches viewed as [Hkv][num_pages * 16 tokens][128]: box {64, 8, Hkv}
+    const uint64_t dims[3] = {static_cast<uint64_t>(kDecD),
+                              static_cast<uint64_t>(num_pages) * kPage,
+                              static_cast<uint64_t>(Hkv)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(Hkv) * kDecD * 2,
+                                 static_cast<uint64_t>(kDecD) * 2};
+    const uint32_t box[3] = {64, static_cast<uint32_t>(kHalf), static_cast<uint32_t>(Hkv)};
+    int rc = encode_tensor_map_16bit(&tmK, kcache, true, 3, dims, strides, box);
+    if (rc == FA_OK) rc = encode_tensor_map_16bit(&tmV, vcache, true, 3, dims, strides, box);
+    if (rc != FA_OK) return rc;
+  } else {
+    memset(&tmK, 0, sizeof(tmK));
+    memset(&tmV, 0, sizeof(tmV));
+  }
   switch (G) {
-    case 1: launch_kernels<1>(prm, pl, stream); break;
-    case 2: launch_kernels<2>(prm, pl, stream); break;
-    case 4: launch_kernels<4>(prm, pl, stream); break;
-    default: launch_kernels<8>(prm, pl, stream); break;
+    case 1: launch_kernels<1>(prm, pl, tmK, tmV, stream); break;
+    case 2: launch_kernels<2>(prm, pl, tmK, tmV, stream); break;
+    case 4: launch_kernels<4>(prm, pl, tmK, tmV, stream); break;
+    default: launch_kernels<8>(prm, pl, tmK, tmV, stream); break;
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(FA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));

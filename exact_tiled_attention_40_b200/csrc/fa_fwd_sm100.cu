@@ -442,43 +442,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult qres;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) ==
-            cudaSuccess &&
-        qres == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  });
-  return fn;
-}
-
 // 3-D map over a contiguous [Z, N, D] tensor of 16-bit elements with a
 // 64 x 128 x 1 box and 128-byte swizzle (one swizzle atom column per box).
 int encode_3d(CUtensorMap* m, const void* base, bool bf16, int D, int N, int Z) {
-  EncodeTiledFn enc = get_encode_fn();
-  if (!enc) return set_error(FA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N),
-                        static_cast<cuuint64_t>(Z)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
-                           static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(D) * 2};
-  cuuint32_t box[3] = {64, 128, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
-                   const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS)
-    return set_error(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", int(r));
-  return FA_OK;
+  const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(N),
+                            static_cast<uint64_t>(Z)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2,
+                               static_cast<uint64_t>(N) * static_cast<uint64_t>(D) * 2};
+  const uint32_t box[3] = {64, 128, 1};
+  return encode_tensor_map_16bit(m, base, bf16, 3, dims, strides, box);
 }
 
 template <int D, bool BF16>

@@ -2,6 +2,7 @@
 #pragma once
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace fa {
@@ -12,6 +13,13 @@ int set_error(int code, const char* fmt, ...);
 // Device pointer of the per-device error word that kernels set on a bounded
 // wait running out or on an out-of-range index read from device memory.
 int* device_error_word(int device);
+
+// Encodes a tiled TMA tensor map over 16-bit elements (bf16 or fp16) with
+// 128-byte swizzle and zero fill.  dims[0] is the contiguous dimension;
+// strides_bytes[i] is the byte stride of dimension i + 1.  Returns an FA_* status.
+int encode_tensor_map_16bit(CUtensorMap* m, const void* base, bool bf16, int rank,
+                            const uint64_t* dims, const uint64_t* strides_bytes,
+                            const uint32_t* box);
 
 // Wall-time limit of every bounded wait inside a kernel.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
