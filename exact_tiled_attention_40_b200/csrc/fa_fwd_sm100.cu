@@ -21,7 +21,8 @@
 //   [  0,128) S0 = Q0 K^T  (its first 64 columns are reused for P0 as bf16 pairs)
 //   [128,256) S1 = Q1 K^T  (P1 likewise)
 //   [256,256+D) O0,  [256+D,256+2D) O1  -- the running unnormalised outputs
-// Per key tile j the MMA thread issues, in order: PV0_j, S0_{j+1}, PV1_j, S1_{j+1}.
+// Per key tile j the MMA thread issues, in order: PV0_j, S0_{j+1}, PV1_j, S1_{j+1},
+// each PV in two halves of 64 keys that the softmax releases as it writes P.
 // tcgen05 operations of one thread execute in issue order, so S_{j+1} never
 // overwrites P_j before PV_j has read it, and the commit that publishes S_{j+1}
 // also guarantees PV_j finished -- the softmax warpgroup may then rescale O in
@@ -63,7 +64,7 @@ struct FwdLayout {
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
-  static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 2 + 2 + 1;
+  static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 4 + 2 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + slack for 1024-byte alignment
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -121,9 +122,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto kv_full = [&](int s) { return bar(2 + s); };
   auto kv_empty = [&](int s) { return bar(2 + L::kSlots + s); };
   auto s_full = [&](int t) { return bar(2 + 2 * L::kSlots + t); };
-  auto p_full = [&](int t) { return bar(4 + 2 * L::kSlots + t); };
-  auto o_full = [&](int t) { return bar(6 + 2 * L::kSlots + t); };
-  const uint32_t mma_done = bar(8 + 2 * L::kSlots);
+  // P is released in two halves (keys 0-63, 64-127) so that the first half of
+  // P V runs while the second half of P is still being computed.
+  auto p_half = [&](int t, int h) { return bar(4 + 2 * L::kSlots + 2 * t + h); };
+  auto o_full = [&](int t) { return bar(8 + 2 * L::kSlots + t); };
+  const uint32_t mma_done = bar(10 + 2 * L::kSlots);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
@@ -131,7 +134,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(q_full(t), 1);
       mbar_init(s_full(t), 1);
-      mbar_init(p_full(t), kBM);
+      mbar_init(p_half(t, 0), kBM);
+      mbar_init(p_half(t, 1), kBM);
       mbar_init(o_full(t), 1);
     }
     for (int s = 0; s < L::kSlots; ++s) {
@@ -220,15 +224,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_commit(s_full(t));
         };
-        // O_t += P_t V : A = P from TMEM (bf16 pairs), B = V tile, MN-major (D contiguous)
-        auto issue_pv = [&](int t, int slot, bool accumulate) {
+        // O_t += P_t V over keys [64 h, 64 h + 64): A = P from TMEM (bf16 pairs),
+        // B = V tile, MN-major (D contiguous)
+        auto issue_pv_half = [&](int t, int slot, int h, bool accumulate) {
           const uint64_t b0 = desc_v + static_cast<uint64_t>((slot * L::kTileBytes) >> 4);
           const uint32_t d = tmem + 256 + t * D;
           const uint32_t a = tmem + t * 128;
   #pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk)
+          for (int k4 = 0; k4 < kBN / 32; ++k4) {
+            const int kk = h * (kBN / 32) + k4;
             mma_ts(d, a + kk * 8, b0 + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_pv,
                    (accumulate || kk > 0) ? 1u : 0u);
+          }
         };
         bool ok = true;
         if (n_kv[0] > 0) ok = mbar_wait(q_full(0), 0, abort_flag, p.err, p.timeout_ns);
@@ -250,10 +257,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   #pragma unroll
           for (int t = 0; t < 2; ++t) {
             if (!ok || j >= (t ? n_kv[1] : n_kv[0])) continue;
-            ok = mbar_wait(p_full(t), j & 1, abort_flag, p.err, p.timeout_ns);
+            ok = mbar_wait(p_half(t, 0), j & 1, abort_flag, p.err, p.timeout_ns);
             if (!ok) continue;
             tc_fence_after();
-            issue_pv(t, slot_of(vpos), j > 0);
+            issue_pv_half(t, slot_of(vpos), 0, j > 0);
+            ok = mbar_wait(p_half(t, 1), j & 1, abort_flag, p.err, p.timeout_ns);
+            if (!ok) continue;
+            tc_fence_after();
+            issue_pv_half(t, slot_of(vpos), 1, true);
             if (j + 1 < (t ? n_kv[1] : n_kv[0]))
               issue_s(t, slot_of(kpos));
             else
@@ -372,6 +383,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               pk[e] = BF16 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
             }
             tmem_st16(tS + 16 * c, pk);
+            if (c == 1) {                        // keys 0-63 of P are in place
+              tmem_wait_st();
+              tc_fence_before();
+              mbar_arrive(p_half(t, 0));
+            }
           }
         } else {
           // unmasked tiles: the first kPolyPairs pairs of every 32 columns on the
@@ -394,6 +410,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               pk[e] = BF16 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
             }
             tmem_st16(tS + 16 * c, pk);
+            if (c == 1) {                        // keys 0-63 of P are in place
+              tmem_wait_st();
+              tc_fence_before();
+              mbar_arrive(p_half(t, 0));
+            }
           }
         }
         float sa, sb;
@@ -401,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         l += sa + sb;
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(p_full(t));
+        mbar_arrive(p_half(t, 1));
       }
       const bool fin = ok && mbar_wait(o_full(t), 0, abort_flag, p.err, p.timeout_ns);
       if (__all_sync(0xffffffffu, fin)) {
