@@ -355,8 +355,9 @@ def main():
         "decode": {"value": dec_gbs, "unit": "GB/s", "kv_bytes_per_step": kv_bytes,
                    "roofline": {"bound": "hbm", "achieved": dec_achieved, "peak": peaks["hbm_gbs"],
                                 "unit": "GB/s", "frac": dec_achieved / peaks["hbm_gbs"],
-                                "traffic": recorded_traffic("fa_decode_split_kernel",
+                                "traffic": recorded_traffic("fa_decode_stream_kernel",
                                                             "fa_decode_sm100.cu"),
+                                "kernel": "fa_decode_paged call: scan + stream<4> + merge",
                                 "peak_source": f"{peak_src} copy bandwidth",
                                 "frac_of_nominal_8000": dec_achieved / 8000.0},
                    "ms_per_launch": statistics.mean(dec_ms)},
@@ -364,7 +365,8 @@ def main():
         "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "what": "prefill through fa_fwd with pinned host "
                 "q,k,v copied in and o,lse copied out inside the timed region"},
-        "gpu_launches": 3 * K,
+        # per step: fa_fwd_kernel, then fa_decode_paged's scan, stream and merge kernels
+        "gpu_launches": 4 * K,
         "clocks": sampler.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
