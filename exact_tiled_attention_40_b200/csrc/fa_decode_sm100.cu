@@ -291,6 +291,7 @@ __host__ __device__ constexpr int stage_kv_bytes(int Hkv) { return 2 * box_bytes
 __global__ void __launch_bounds__(1024) fa_decode_scan_kernel(const DecodeParams p) {
   __shared__ int warp_sums[32];
   __shared__ int carry;
+  pdl_launch_dependents();   // the stream kernel may launch now; it waits for hb itself
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) carry = 0;
   __syncthreads();
@@ -358,14 +359,9 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   __shared__ StageMeta meta[kMaxStages];
   __shared__ int abort_sm;
 
+  pdl_launch_dependents();   // the merge kernel may launch now; it waits for this grid
   const int c = blockIdx.x;
   const int C = gridDim.x;
-  const int H = p.hb[p.B];
-  const int x0 = static_cast<int>((static_cast<long long>(c) * H) / C);
-  const int x1 = static_cast<int>((static_cast<long long>(c + 1) * H) / C);
-  const int n = x1 - x0;
-  if (n <= 0) return;                          // the same for every thread of the CTA
-
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int NS = p.nstages;
@@ -384,6 +380,13 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     abort_sm = 0;
     fence_barrier_init();
   }
+  // Everything above overlaps the scan kernel; the half-page offsets are its output.
+  pdl_wait();
+  const int H = p.hb[p.B];
+  const int x0 = static_cast<int>((static_cast<long long>(c) * H) / C);
+  const int x1 = static_cast<int>((static_cast<long long>(c + 1) * H) / C);
+  const int n = x1 - x0;
+  if (n <= 0) return;                          // the same for every thread of the CTA
   __syncthreads();
 
   if (warp >= kConsumerWarps) {
@@ -572,6 +575,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
 // half-page list meets b; they are merged by their LSE (formula 2 of the
 // softmax merge).  Lane i owns output columns [4i, 4i + 4).
 __global__ void __launch_bounds__(128) fa_decode_stream_merge_kernel(const DecodeParams p) {
+  pdl_wait();                                  // the stream kernel's partials
   const int wid = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (wid >= p.B * p.Hq) return;
@@ -728,24 +732,50 @@ DecodePlan make_plan(int B, int Hq, int Hkv, int max_pages_per_seq, int nsm) {
 }
 
 template <int G>
-void launch_kernels(const DecodeParams& prm, const DecodePlan& pl, const CUtensorMap& tmK,
-                    const CUtensorMap& tmV, cudaStream_t stream) {
+int launch_kernels(const DecodeParams& prm, const DecodePlan& pl, const CUtensorMap& tmK,
+                   const CUtensorMap& tmV, cudaStream_t stream, int device) {
   if (pl.streamed) {
     const int smem = pl.nstages * 2 * stage_kv_bytes(prm.Hkv) + 1024;
-    static bool attr_done = false;   // the attribute belongs to the function, per process
-    if (!attr_done) {
-      cudaFuncSetAttribute(fa_decode_stream_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kStreamSmemBudget + 1024);
-      attr_done = true;
+    {
+      // the shared-memory limit is a property of the function on each device
+      static bool attr_done[64] = {};
+      static std::mutex mu;
+      std::lock_guard<std::mutex> g(mu);
+      if (device < 0 || device >= 64) return set_error(FA_ERR_CUDA, "device ordinal out of range");
+      if (!attr_done[device]) {
+        cudaError_t e = cudaFuncSetAttribute(fa_decode_stream_kernel<G>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kStreamSmemBudget + 1024);
+        if (e != cudaSuccess)
+          return set_error(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        attr_done[device] = true;
+      }
     }
+    // The stream and merge kernels are launched with programmatic serialization:
+    // each may start while its predecessor runs and waits (griddepcontrol.wait)
+    // before it reads the predecessor's output, which hides the launch gaps.
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.stream = stream;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
     fa_decode_scan_kernel<<<1, 1024, 0, stream>>>(prm);
-    fa_decode_stream_kernel<G><<<pl.nctas, kStreamThreads, smem, stream>>>(tmK, tmV, prm);
-    fa_decode_stream_merge_kernel<<<(prm.B * prm.Hq + 3) / 4, 128, 0, stream>>>(prm);
+    cfg.gridDim = dim3(pl.nctas);
+    cfg.blockDim = dim3(kStreamThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchKernelEx(&cfg, fa_decode_stream_kernel<G>, tmK, tmV, prm);
+    cfg.gridDim = dim3((prm.B * prm.Hq + 3) / 4);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cudaLaunchKernelEx(&cfg, fa_decode_stream_merge_kernel, prm);
   } else {
     dim3 grid(pl.nsplit, prm.B);
     fa_decode_split_kernel<G><<<grid, kDecThreads, 0, stream>>>(prm);
     fa_decode_combine_kernel<<<prm.B * prm.Hq, kDecD, 0, stream>>>(prm);
   }
+  return FA_OK;
 }
 
 // Runs one decode with the given workspace (at least pl.bytes, 256-byte aligned).
@@ -797,12 +827,14 @@ int run_decode(const void* q, const void* kcache, const void* vcache, const int3
     memset(&tmK, 0, sizeof(tmK));
     memset(&tmV, 0, sizeof(tmV));
   }
+  int lrc;
   switch (G) {
-    case 1: launch_kernels<1>(prm, pl, tmK, tmV, stream); break;
-    case 2: launch_kernels<2>(prm, pl, tmK, tmV, stream); break;
-    case 4: launch_kernels<4>(prm, pl, tmK, tmV, stream); break;
-    default: launch_kernels<8>(prm, pl, tmK, tmV, stream); break;
+    case 1: lrc = launch_kernels<1>(prm, pl, tmK, tmV, stream, device); break;
+    case 2: lrc = launch_kernels<2>(prm, pl, tmK, tmV, stream, device); break;
+    case 4: lrc = launch_kernels<4>(prm, pl, tmK, tmV, stream, device); break;
+    default: lrc = launch_kernels<8>(prm, pl, tmK, tmV, stream, device); break;
   }
+  if (lrc != FA_OK) return lrc;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(FA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
   return FA_OK;

@@ -60,7 +60,7 @@ struct FwdLayout {
   static constexpr int kChunks = D / 64;              // 128-byte swizzle atoms along D
   static constexpr int kChunkBytes = kBM * 128;       // one atom column of a 128-row tile
   static constexpr int kTileBytes = kBM * D * 2;      // a 128-row tile of Q, K or V
-  static constexpr int kSlots = D == 128 ? 4 : 8;     // K/V ring slots
+  static constexpr int kSlots = D == 128 ? 5 : 8;     // K/V ring slots
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
@@ -201,11 +201,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (warp == 9) {
       // ------------------------------------------------------------ MMA issuer
-      if (lane == 0 && n_max > 0) {
+      // The whole warp runs the waits, loop counters and descriptor arithmetic
+      // (all warp-uniform); one elected lane issues the MMAs and commits.
+      if (n_max > 0) {
+        const bool leader = elect_one();
         constexpr uint32_t idesc_s = idesc_f16(kBM, kBN, BF16, false);
         constexpr uint32_t idesc_pv = idesc_f16(kBM, D, BF16, true);
         auto slot_of = [&](int pos) { return pos % L::kSlots; };
         auto phase_of = [&](int pos) { return static_cast<uint32_t>((pos / L::kSlots) & 1); };
+        auto wait = [&](uint32_t bar, uint32_t parity) {
+          return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.err, p.timeout_ns));
+        };
+        auto commit = [&](uint32_t bar) {
+          if (leader) tc_commit(bar);
+        };
         // Descriptors are built once; moving to another K step or ring slot only
         // adds (byte offset >> 4) to the start-address field in the low bits.
         const uint64_t desc_q0 = smem_desc_sw128(sbase + L::kQOff, 16, 1024);
@@ -217,12 +226,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t a0 = t ? desc_q1 : desc_q0;
           const uint64_t b0 = desc_k + static_cast<uint64_t>((slot * L::kTileBytes) >> 4);
           const uint32_t d = tmem + t * 128;
+          if (leader) {
   #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * L::kChunkBytes + (kk & 3) * 32) >> 4);
-            mma_ss(d, a0 + off, b0 + off, idesc_s, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t off =
+                  static_cast<uint64_t>(((kk >> 2) * L::kChunkBytes + (kk & 3) * 32) >> 4);
+              mma_ss(d, a0 + off, b0 + off, idesc_s, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(s_full(t));
           }
-          tc_commit(s_full(t));
         };
         // O_t += P_t V over keys [64 h, 64 h + 64): A = P from TMEM (bf16 pairs),
         // B = V tile, MN-major (D contiguous)
@@ -230,56 +242,64 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t b0 = desc_v + static_cast<uint64_t>((slot * L::kTileBytes) >> 4);
           const uint32_t d = tmem + 256 + t * D;
           const uint32_t a = tmem + t * 128;
+          if (leader) {
   #pragma unroll
-          for (int k4 = 0; k4 < kBN / 32; ++k4) {
-            const int kk = h * (kBN / 32) + k4;
-            mma_ts(d, a + kk * 8, b0 + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_pv,
-                   (accumulate || kk > 0) ? 1u : 0u);
+            for (int k4 = 0; k4 < kBN / 32; ++k4) {
+              const int kk = h * (kBN / 32) + k4;
+              mma_ts(d, a + kk * 8, b0 + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_pv,
+                     (accumulate || kk > 0) ? 1u : 0u);
+            }
           }
         };
         bool ok = true;
-        if (n_kv[0] > 0) ok = mbar_wait(q_full(0), 0, abort_flag, p.err, p.timeout_ns);
-        if (ok && n_kv[1] > 0) ok = mbar_wait(q_full(1), 0, abort_flag, p.err, p.timeout_ns);
-        if (ok) ok = mbar_wait(kv_full(slot_of(0)), phase_of(0), abort_flag, p.err, p.timeout_ns);
+        if (n_kv[0] > 0) ok = wait(q_full(0), 0);
+        if (ok && n_kv[1] > 0) ok = wait(q_full(1), 0);
+        if (ok) ok = wait(kv_full(slot_of(0)), phase_of(0));
         if (ok) {
           tc_fence_after();
           if (n_kv[0] > 0) issue_s(0, slot_of(0));
           if (n_kv[1] > 0) issue_s(1, slot_of(0));
-          tc_commit(kv_empty(slot_of(0)));
+          commit(kv_empty(slot_of(0)));
         }
         for (int j = 0; j < n_max && ok; ++j) {
           const int vpos = 2 * j + 1;
           const int kpos = 2 * j + 2;
           const bool has_next = j + 1 < n_max;
-          ok = mbar_wait(kv_full(slot_of(vpos)), phase_of(vpos), abort_flag, p.err, p.timeout_ns);
-          if (ok && has_next)
-            ok = mbar_wait(kv_full(slot_of(kpos)), phase_of(kpos), abort_flag, p.err, p.timeout_ns);
+          ok = wait(kv_full(slot_of(vpos)), phase_of(vpos));
+          bool k_ready = false;   // K_{j+1} is waited for just before its first use
   #pragma unroll
           for (int t = 0; t < 2; ++t) {
             if (!ok || j >= (t ? n_kv[1] : n_kv[0])) continue;
-            ok = mbar_wait(p_half(t, 0), j & 1, abort_flag, p.err, p.timeout_ns);
+            ok = wait(p_half(t, 0), j & 1);
             if (!ok) continue;
             tc_fence_after();
             issue_pv_half(t, slot_of(vpos), 0, j > 0);
-            ok = mbar_wait(p_half(t, 1), j & 1, abort_flag, p.err, p.timeout_ns);
+            ok = wait(p_half(t, 1), j & 1);
             if (!ok) continue;
             tc_fence_after();
             issue_pv_half(t, slot_of(vpos), 1, true);
-            if (j + 1 < (t ? n_kv[1] : n_kv[0]))
+            if (j + 1 < (t ? n_kv[1] : n_kv[0])) {
+              if (!k_ready) {
+                ok = wait(kv_full(slot_of(kpos)), phase_of(kpos));
+                k_ready = true;
+                if (!ok) continue;
+                tc_fence_after();
+              }
               issue_s(t, slot_of(kpos));
-            else
-              tc_commit(o_full(t));
+            } else {
+              commit(o_full(t));
+            }
           }
           if (!ok) break;
-          tc_commit(kv_empty(slot_of(vpos)));
-          if (has_next) tc_commit(kv_empty(slot_of(kpos)));
+          commit(kv_empty(slot_of(vpos)));
+          if (has_next) commit(kv_empty(slot_of(kpos)));
         }
         // All issued MMAs must complete before TMEM is released (also on abort).
-        tc_commit(mma_done);
+        commit(mma_done);
         volatile int no_abort = 0;
         mbar_wait(mma_done, 0, &no_abort, p.err, p.timeout_ns);
       }
-  }
+    }
   } else {
     regs_inc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax warpgroups

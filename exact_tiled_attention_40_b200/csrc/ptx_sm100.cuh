@@ -143,6 +143,27 @@ __device__ __forceinline__ void tc_fence_after() {
 }
 // Arrive once on `bar` when every tcgen05 operation issued so far by this
 // thread has completed.
+// Programmatic dependent launch.  pdl_launch_dependents lets the next kernel of
+// the stream begin launching while this one runs; pdl_wait blocks until the
+// kernels this one depends on have completed and their writes are visible.
+// Both are no-ops for a kernel launched without programmatic serialization.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// True in exactly one lane (the lowest) of a converged warp; every lane of the
+// warp must execute it.  Lets a whole warp run the control flow of a
+// single-thread issuer (waits, loop counters, descriptor arithmetic) while one
+// lane issues the instructions.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
