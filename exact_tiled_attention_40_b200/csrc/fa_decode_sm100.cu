@@ -33,6 +33,7 @@
 //    straight from HBM with 16-byte non-allocating loads.
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 #include <vector>
 
@@ -57,11 +58,24 @@ constexpr int kStreamThreads = 12 * 32;          // 8 consumer warps + a produce
 // Register split (setmaxnreg): the producer warpgroup (warps 8-11, one of them
 // working) gives registers to the two consumer warpgroups; 40 x 128 + 224 x 256
 // stays within the 384 x 168 the block is launched with.
-constexpr uint32_t kRegsProducer = 40;
+constexpr uint32_t kRegsProducer = 48;
 constexpr uint32_t kRegsConsumer = 224;
 static_assert(kRegsProducer * 128 + kRegsConsumer * 256 <= 384 * 168, "register split");
 constexpr int kMaxStages = 8;
 constexpr int kStreamSmemBudget = 200 * 1024;
+// Streamed schedule: the half-page list is split into equal contiguous shares,
+// one per CTA.  The first ~90 % of each share is streamed by its own CTA; the
+// last tenth is cut into units of kDynUnit half-pages that go to whichever CTA
+// asks first, so CTAs that stream more slowly (SMs differ in the bandwidth they
+// get) finish with the others.  Keeping each share's units next to it spreads
+// them over all sequences, so no sequence collects many partials.
+constexpr int kDynDiv = 10;    // 1 / kDynDiv of each share is dynamic
+constexpr int kDynUnit = 8;    // half-pages per dynamic unit (at least)
+constexpr int kMaxUnitsPerCta = 4;
+constexpr int kMaxStreamCtas = 204;                       // so a sequence has <= 1024 partials
+constexpr int kMaxMergeSlots = kMaxStreamCtas * (1 + kMaxUnitsPerCta);
+constexpr int kMergeWarps = 32;
+constexpr int kHbSmemMax = 4096;   // sequences whose offsets the producer keeps in shared memory
 
 struct DecodeParams {
   const uint16_t* q;
@@ -74,9 +88,12 @@ struct DecodeParams {
   float* ws_o;     // partial outputs, [slot][Hq][128] normalised
   float* ws_lse;   // partial LSE (natural log), [slot][Hq]
   int* hb;         // streamed: hb[b] = half-pages before sequence b, hb[B] = total
+  int* dyn_next;   // streamed: next dynamic unit to hand out (zeroed by the scan kernel)
   int B, Hq, Hkv, max_pages, num_pages;
   int pps, nsplit;             // direct schedule
   int nctas, nstages;          // streamed schedule
+  int dyn_units_cap;           // streamed: partial slots reserved for dynamic units
+  int hb_in_smem;              // streamed: the producer copies hb to shared memory
   float scale_log2;
   int* err;
 };
@@ -293,7 +310,10 @@ __global__ void __launch_bounds__(1024) fa_decode_scan_kernel(const DecodeParams
   __shared__ int carry;
   pdl_launch_dependents();   // the stream kernel may launch now; it waits for hb itself
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (threadIdx.x == 0) carry = 0;
+  if (threadIdx.x == 0) {
+    carry = 0;
+    *p.dyn_next = 0;
+  }
   __syncthreads();
   for (int base = 0; base < p.B; base += 1024) {
     const int b = base + threadIdx.x;
@@ -332,17 +352,59 @@ __global__ void __launch_bounds__(1024) fa_decode_scan_kernel(const DecodeParams
   if (threadIdx.x == 0) p.hb[p.B] = carry;
 }
 
-// CTA c's share of the H half-pages is [c*H/C, (c+1)*H/C); it may be empty.
-__device__ __forceinline__ bool share_nonempty(long long c, long long H, long long C) {
-  return ((c + 1) * H) / C > (c * H) / C;
-}
-// CTA holding half-page x: the largest c with c*H/C <= x.
+// CTA whose share [c*H/C, (c+1)*H/C) holds half-page x < H: the largest c with
+// c*H/C <= x.
 __device__ __forceinline__ int cta_of(long long x, long long H, long long C) {
+  if ((x + 1) * C <= 0x7fffffffLL)             // the usual case: 32-bit division
+    return static_cast<int>((static_cast<uint32_t>(x + 1) * static_cast<uint32_t>(C) - 1u) /
+                            static_cast<uint32_t>(H));
   return static_cast<int>(((x + 1) * C - 1) / H);
+}
+// floor(c * H / C) for 0 <= c <= C
+__device__ __forceinline__ int share_edge(int c, int H, int C) {
+  const long long prod = static_cast<long long>(c) * H;
+  if (prod <= 0x7fffffffLL)
+    return static_cast<int>(static_cast<uint32_t>(prod) / static_cast<uint32_t>(C));
+  return static_cast<int>(prod / C);
+}
+
+// Share of CTA c: [x0, x1) = [c*H/C, (c+1)*H/C); its own part [x0, y) and its
+// dynamic part [y, x1) of d = (x1 - x0) / kDynDiv half-pages, cut into units of
+// U half-pages; unit k of CTA c is global unit c * NUc + k (it may be empty).
+// At most cap units in all (cap < C: no dynamic parts).  The partial of a
+// segment of sequence b goes to slot c + b (own part of CTA c) or
+// C + B + u + b (unit u): along the list the sequence index and the share or
+// unit index never both stay the same, so the slots are distinct.
+struct StreamSplit {
+  int U, NUc;
+};
+__device__ __forceinline__ StreamSplit stream_split(int H, int C, int cap) {
+  StreamSplit sp;
+  sp.U = kDynUnit;
+  sp.NUc = 0;
+  const int per_cta = min(cap / C, kMaxUnitsPerCta);
+  const int dmax = ((H + C - 1) / C) / kDynDiv;
+  if (per_cta > 0 && dmax > 0) {
+    if ((dmax + sp.U - 1) / sp.U > per_cta) sp.U = (dmax + per_cta - 1) / per_cta;
+    sp.NUc = (dmax + sp.U - 1) / sp.U;
+  }
+  return sp;
+}
+struct Share {
+  int x0, y, x1;
+};
+__device__ __forceinline__ Share share_of(int c, int H, int C, const StreamSplit& sp) {
+  Share sh;
+  sh.x0 = share_edge(c, H, C);
+  sh.x1 = share_edge(c + 1, H, C);
+  sh.y = sh.x1 - (sp.NUc > 0 ? (sh.x1 - sh.x0) / kDynDiv : 0);
+  return sh;
 }
 
 struct StageMeta {
-  int b, hh, flags, len;   // flags: 1 = first of segment, 2 = last of segment, 4 = page valid
+  int b, hh, flags, len;   // flags: 1 = first of segment, 2 = last of segment, 4 = page valid,
+                           //        8 = no more stages
+  int slot0;               // partial slot of this segment = slot0 + b
 };
 
 template <int G>
@@ -383,78 +445,116 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   // Everything above overlaps the scan kernel; the half-page offsets are its output.
   pdl_wait();
   const int H = p.hb[p.B];
-  const int x0 = static_cast<int>((static_cast<long long>(c) * H) / C);
-  const int x1 = static_cast<int>((static_cast<long long>(c + 1) * H) / C);
-  const int n = x1 - x0;
-  if (n <= 0) return;                          // the same for every thread of the CTA
+  const StreamSplit sp = stream_split(H, C, p.dyn_units_cap);
+  const Share own = share_of(c, H, C, sp);
   __syncthreads();
 
   if (warp >= kConsumerWarps) {
     regs_dec<kRegsProducer>();
     if (warp != kConsumerWarps) return;
     // ---------------------------------------------------------------- producer
-    // The whole warp resolves the next 32 stages (sequence, half-page, page id,
-    // length) with independent loads; lane 0 then issues them in order.
+    // The sequence offsets are searched for every stage: keep them in shared
+    // memory (after the stage ring) when they fit.
+    const int* hbp = p.hb;
+    if (p.hb_in_smem) {
+      int* hb_sm = reinterpret_cast<int*>(dsm_raw + (sbase - smem_u32(dsm_raw)) + NS * 2 * SKV);
+      for (int i = lane; i <= p.B; i += 32) hb_sm[i] = p.hb[i];
+      __syncwarp();
+      hbp = hb_sm;
+    }
+    // Ranges of the half-page list: this CTA's static share, then dynamic units
+    // while any are left.  For each range the whole warp resolves the next 32
+    // stages (sequence, half-page, page id, length) with independent loads and
+    // lane 0 issues them in order.  A last stage flagged 8 ends the consumers.
     int issued = 0;
     bool ok = true;
-    for (int base = 0; base < n && ok; base += 32) {
-      const int i = base + lane;
-      int bq = 0, hh = 0, page = -1, len = 0, flags = 0;
-      if (i < n) {
-        const int x = x0 + i;
-        int lo = 0, hi = p.B;                  // hb[lo] <= x < hb[hi]
-        while (hi - lo > 1) {
-          const int mid = (lo + hi) >> 1;
-          if (p.hb[mid] <= x) lo = mid; else hi = mid;
-        }
-        bq = lo;
-        const int hb_b = p.hb[bq], hb_n = p.hb[bq + 1];
-        hh = x - hb_b;
-        page = p.block_table[static_cast<size_t>(bq) * p.max_pages + (hh >> 1)];
-        len = p.seq_lens[bq];
-        const bool valid = page >= 0 && page < p.num_pages;
-        flags = ((i == 0 || hh == 0) ? 1 : 0) | ((i == n - 1 || x + 1 == hb_n) ? 2 : 0) |
-                (valid ? 4 : 0);
-      }
-      const int cnt_here = min(32, n - base);
-      for (int k = 0; k < cnt_here; ++k) {
-        const int kb = __shfl_sync(0xffffffffu, bq, k);
-        const int khh = __shfl_sync(0xffffffffu, hh, k);
-        const int kpage = __shfl_sync(0xffffffffu, page, k);
-        const int klen = __shfl_sync(0xffffffffu, len, k);
-        const int kflags = __shfl_sync(0xffffffffu, flags, k);
-        if (lane == 0) {
-          const int ii = base + k;
-          const int st = ii % NS;
-          if (!mbar_wait_sleepy(empty(st), ((ii / NS) & 1) ^ 1, abort_flag, p.err, kWaitLimitNs)) {
-            ok = false;
-          } else {
-            StageMeta md;
-            md.b = kb;
-            md.hh = khh;
-            md.len = klen;
-            md.flags = kflags;
-            meta[st] = md;
-            if (kflags & 4) {
-              const int tok0 = kpage * kPage + (khh & 1) * kHalf;
-              const uint32_t kdst = sbase + st * 2 * SKV;
-              mbar_arrive_expect_tx(full(st), 2 * SKV);
-              tma_load_3d(kdst, &tmK, full(st), 0, tok0, 0);
-              tma_load_3d(kdst + HB, &tmK, full(st), 64, tok0, 0);
-              tma_load_3d(kdst + SKV, &tmV, full(st), 0, tok0, 0);
-              tma_load_3d(kdst + SKV + HB, &tmV, full(st), 64, tok0, 0);
-            } else {
-              atomicOr(p.err, kErrBadIndex);   // consumers skip this stage
-              mbar_arrive(full(st));
-            }
-            ++issued;
+    auto acquire_stage = [&](int& st) {
+      st = issued % NS;
+      return mbar_wait_sleepy(empty(st), ((issued / NS) & 1) ^ 1, abort_flag, p.err, kWaitLimitNs);
+    };
+    auto run_range = [&](int xs, int cnt, int slot0) {
+      for (int base = 0; base < cnt && ok; base += 32) {
+        const int i = base + lane;
+        int bq = 0, hh = 0, page = -1, len = 0, flags = 0;
+        if (i < cnt) {
+          const int x = xs + i;
+          int lo = 0, hi = p.B;                  // hb[lo] <= x < hb[hi]
+          while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (hbp[mid] <= x) lo = mid; else hi = mid;
           }
+          bq = lo;
+          const int hb_b = hbp[bq], hb_n = hbp[bq + 1];
+          hh = x - hb_b;
+          page = p.block_table[static_cast<size_t>(bq) * p.max_pages + (hh >> 1)];
+          len = p.seq_lens[bq];
+          const bool valid = page >= 0 && page < p.num_pages;
+          flags = ((i == 0 || hh == 0) ? 1 : 0) | ((i == cnt - 1 || x + 1 == hb_n) ? 2 : 0) |
+                  (valid ? 4 : 0);
         }
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        if (!ok) break;
+        const int cnt_here = min(32, cnt - base);
+        for (int k = 0; k < cnt_here; ++k) {
+          const int kb = __shfl_sync(0xffffffffu, bq, k);
+          const int khh = __shfl_sync(0xffffffffu, hh, k);
+          const int kpage = __shfl_sync(0xffffffffu, page, k);
+          const int klen = __shfl_sync(0xffffffffu, len, k);
+          const int kflags = __shfl_sync(0xffffffffu, flags, k);
+          if (lane == 0) {
+            int st;
+            if (!acquire_stage(st)) {
+              ok = false;
+            } else {
+              StageMeta md;
+              md.b = kb;
+              md.hh = khh;
+              md.len = klen;
+              md.flags = kflags;
+              md.slot0 = slot0;
+              meta[st] = md;
+              if (kflags & 4) {
+                const int tok0 = kpage * kPage + (khh & 1) * kHalf;
+                const uint32_t kdst = sbase + st * 2 * SKV;
+                mbar_arrive_expect_tx(full(st), 2 * SKV);
+                tma_load_3d(kdst, &tmK, full(st), 0, tok0, 0);
+                tma_load_3d(kdst + HB, &tmK, full(st), 64, tok0, 0);
+                tma_load_3d(kdst + SKV, &tmV, full(st), 0, tok0, 0);
+                tma_load_3d(kdst + SKV + HB, &tmV, full(st), 64, tok0, 0);
+              } else {
+                atomicOr(p.err, kErrBadIndex);   // consumers skip this stage
+                mbar_arrive(full(st));
+              }
+              ++issued;
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
+        }
       }
+    };
+    if (own.y > own.x0) run_range(own.x0, own.y - own.x0, c);
+    const int n_units = C * sp.NUc;
+    while (ok && n_units > 0) {
+      int u = 0;
+      if (lane == 0) u = atomicAdd(p.dyn_next, 1);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      if (u >= n_units) break;
+      const Share sh = share_of(u / sp.NUc, H, C, sp);
+      const int xs = sh.y + (u % sp.NUc) * sp.U;
+      if (xs < sh.x1) run_range(xs, min(sh.x1, xs + sp.U) - xs, C + p.B + u);
     }
     if (lane == 0) {
+      int st;
+      if (ok && acquire_stage(st)) {             // end marker: no copy behind it
+        StageMeta md;
+        md.b = 0;
+        md.hh = 0;
+        md.len = 0;
+        md.flags = 8;
+        md.slot0 = 0;
+        meta[st] = md;
+        mbar_arrive(full(st));
+        ++issued;
+      }
       // copies still in flight must land before the CTA exits
       volatile int no_abort = 0;
       for (int i = max(0, issued - NS); i < issued; ++i)
@@ -488,11 +588,12 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   for (int dg = 0; dg < 4; ++dg)
     ld_off[dg] = static_cast<uint32_t>((dg >> 1) * HB) + row_off +
                  static_cast<uint32_t>((((dg & 1) * 4 + (lane >> 3)) ^ lt) << 4);
-  for (int i = 0; i < n; ++i) {
+  for (int i = 0;; ++i) {
     const int st = i % NS;
     const bool ready = mbar_wait(full(st), (i / NS) & 1, abort_flag, p.err, kWaitLimitNs);
     if (!__all_sync(0xffffffffu, ready)) return;
     const StageMeta md = meta[st];
+    if (md.flags & 8) break;                   // the producer has no more stages
     if (active) {
       if (md.flags & 1) {                      // a new sequence segment begins
         m_run = -INFINITY;
@@ -549,13 +650,13 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
         }
       }
 
-      if (md.flags & 2) {                      // segment ends: write its partial to slot c + b
+      if (md.flags & 2) {                      // segment ends: its partial goes to slot0 + b
         float l_tot = l_run;
         l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 1);
         l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 2);
         if (my_row) {
           const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
-          const size_t rowi = (static_cast<size_t>(c) + md.b) * p.Hq + hq;
+          const size_t rowi = (static_cast<size_t>(md.slot0) + md.b) * p.Hq + hq;
           float* dst = p.ws_o + rowi * kDecD + 2 * tq;
 #pragma unroll
           for (int nn = 0; nn < 16; ++nn)
@@ -570,51 +671,104 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   }
 }
 
-// Streamed schedule, merge: one warp per (sequence b, query head h).  The
-// partials of b sit in slots c + b for every CTA c whose non-empty share of the
-// half-page list meets b; they are merged by their LSE (formula 2 of the
-// softmax merge).  Lane i owns output columns [4i, 4i + 4).
-__global__ void __launch_bounds__(128) fa_decode_stream_merge_kernel(const DecodeParams p) {
+// Streamed schedule, merge: one block per sequence b.  The partials of b sit in
+// slot c + b for every CTA c whose own part meets b, and in slot C + B + u + b
+// for every dynamic unit u that meets b; warp 0 lists them in shared memory
+// (lanes over CTAs), then each warp merges query heads by their LSE (formula 2
+// of the softmax merge), lane i owning output columns [4i, 4i + 4).
+__global__ void __launch_bounds__(kMergeWarps * 32) fa_decode_stream_merge_kernel(
+    const DecodeParams p) {
+  __shared__ int slots[kMaxMergeSlots];
+  __shared__ int n_slots_sm;
   pdl_wait();                                  // the stream kernel's partials
-  const int wid = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  if (wid >= p.B * p.Hq) return;
-  const int b = wid / p.Hq;
-  const int h = wid - b * p.Hq;
   const int xs = p.hb[b], xe = p.hb[b + 1];
   if (xe <= xs) {                              // no keys (or an invalid length): O = 0, LSE = -inf
-    *reinterpret_cast<uint2*>(p.o + static_cast<size_t>(wid) * kDecD + lane * 4) = make_uint2(0, 0);
-    if (p.lse && lane == 0) p.lse[wid] = -INFINITY;
+    for (int h = warp; h < p.Hq; h += kMergeWarps) {
+      const size_t wid = static_cast<size_t>(b) * p.Hq + h;
+      *reinterpret_cast<uint2*>(p.o + wid * kDecD + lane * 4) = make_uint2(0, 0);
+      if (p.lse && lane == 0) p.lse[wid] = -INFINITY;
+    }
     return;
   }
-  const long long H = p.hb[p.B], C = p.nctas;
-  const int c_first = cta_of(xs, H, C), c_last = cta_of(xe - 1, H, C);
-  // lane-parallel LSE pass over the (few) contributing CTAs
-  float mx = -INFINITY;
-  for (int cc = c_first + lane; cc <= c_last; cc += 32)
-    if (share_nonempty(cc, H, C)) mx = fmaxf(mx, p.ws_lse[(static_cast<size_t>(cc) + b) * p.Hq + h]);
+  const int H = p.hb[p.B];
+  const int C = p.nctas;
+  const StreamSplit sp = stream_split(H, C, p.dyn_units_cap);
+  if (warp == 0) {
+    const int c_first = cta_of(xs, H, C), c_last = cta_of(xe - 1, H, C);
+    int base = 0;
+    for (int c0 = c_first; c0 <= c_last; c0 += 32) {
+      const int cc = c0 + lane;
+      Share sh;
+      int own = 0, k0 = 0, k1 = -1;
+      if (cc <= c_last) {
+        sh = share_of(cc, H, C, sp);
+        own = max(xs, sh.x0) < min(xe, sh.y) ? 1 : 0;
+        const int lo = max(xs, sh.y), hi = min(xe, sh.x1);
+        if (lo < hi) {
+          k0 = (lo - sh.y) / sp.U;
+          k1 = (hi - 1 - sh.y) / sp.U;
+        }
+      }
+      const int cnt = own + (k1 - k0 + 1);
+      int incl = cnt;                          // inclusive prefix over the lanes
 #pragma unroll
-  for (int d = 16; d >= 1; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
-  float wsum = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (mx > -INFINITY) {
-    for (int cc = c_first; cc <= c_last; ++cc) {
-      if (!share_nonempty(cc, H, C)) continue;
-      const size_t row = (static_cast<size_t>(cc) + b) * p.Hq + h;
-      const float ls = p.ws_lse[row];
-      const float w = (ls == -INFINITY) ? 0.f : ex2((ls - mx) * kLog2e);
-      wsum += w;
-      const float4 v = reinterpret_cast<const float4*>(p.ws_o + row * kDecD)[lane];
-      acc.x = fmaf(w, v.x, acc.x);
-      acc.y = fmaf(w, v.y, acc.y);
-      acc.z = fmaf(w, v.z, acc.z);
-      acc.w = fmaf(w, v.w, acc.w);
+      for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += y;
+      }
+      int at = base + incl - cnt;
+      if (own && at < kMaxMergeSlots) slots[at] = cc + b;
+      at += own;
+      for (int k = k0; k <= k1; ++k, ++at)
+        if (at < kMaxMergeSlots) slots[at] = C + p.B + cc * sp.NUc + k + b;
+      base += __shfl_sync(0xffffffffu, incl, 31);
     }
+    if (lane == 0) n_slots_sm = min(base, kMaxMergeSlots);
   }
-  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-  *reinterpret_cast<uint2*>(p.o + static_cast<size_t>(wid) * kDecD + lane * 4) =
-      make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
-  if (p.lse && lane == 0) p.lse[wid] = wsum > 0.f ? mx + __log2f(wsum) * kLn2 : -INFINITY;
+  __syncthreads();
+  const int ns = n_slots_sm;
+  for (int h = warp; h < p.Hq; h += kMergeWarps) {
+    float mx = -INFINITY;
+    for (int k = lane; k < ns; k += 32)
+      mx = fmaxf(mx, p.ws_lse[static_cast<size_t>(slots[k]) * p.Hq + h]);
+#pragma unroll
+    for (int d = 16; d >= 1; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
+    float wsum = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (mx > -INFINITY) {
+      // weights lane-parallel, 32 slots at a time; each lane then accumulates its
+      // four columns over those slots with independent loads
+      for (int k0 = 0; k0 < ns; k0 += 32) {
+        float w = 0.f;
+        if (k0 + lane < ns) {
+          const float ls = p.ws_lse[static_cast<size_t>(slots[k0 + lane]) * p.Hq + h];
+          w = (ls == -INFINITY) ? 0.f : ex2((ls - mx) * kLog2e);
+        }
+        wsum += w;
+        const int cnt = min(32, ns - k0);
+#pragma unroll 8
+        for (int j = 0; j < cnt; ++j) {
+          const float wj = __shfl_sync(0xffffffffu, w, j);
+          const size_t row = static_cast<size_t>(slots[k0 + j]) * p.Hq + h;
+          const float4 v = reinterpret_cast<const float4*>(p.ws_o + row * kDecD)[lane];
+          acc.x = fmaf(wj, v.x, acc.x);
+          acc.y = fmaf(wj, v.y, acc.y);
+          acc.z = fmaf(wj, v.z, acc.z);
+          acc.w = fmaf(wj, v.w, acc.w);
+        }
+      }
+#pragma unroll
+      for (int d = 16; d >= 1; d >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, d);
+    }
+    const size_t wid = static_cast<size_t>(b) * p.Hq + h;
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    *reinterpret_cast<uint2*>(p.o + wid * kDecD + lane * 4) =
+        make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
+    if (p.lse && lane == 0) p.lse[wid] = wsum > 0.f ? mx + __log2f(wsum) * kLn2 : -INFINITY;
+  }
 }
 
 // One CTA of 128 threads per (sequence, query head); thread d owns output column d.
@@ -693,6 +847,7 @@ struct DecodePlan {
   bool streamed = false;
   int pps = 0, nsplit = 0;     // direct schedule
   int nctas = 0, nstages = 0;  // streamed schedule
+  int dyn_units_cap = 0;       // streamed: dynamic units the partial slots allow
   size_t n_part = 0;           // partial rows (slot x head)
   size_t bytes = 0;            // workspace bytes
 };
@@ -707,8 +862,10 @@ int direct_pps(int B, int max_pages_per_seq) {
 
 void finish_plan(DecodePlan& pl, int B, int Hq, int Hkv) {
   if (pl.streamed) {
-    pl.n_part = (static_cast<size_t>(pl.nctas) + B) * Hq;
-    pl.bytes = pl.n_part * (kDecD + 1) * sizeof(float) + (static_cast<size_t>(B) + 1) * sizeof(int);
+    // slots: C + B static, then (units + B) dynamic when there are units
+    const size_t dyn_slots = pl.dyn_units_cap > 0 ? static_cast<size_t>(pl.dyn_units_cap) + B : 0;
+    pl.n_part = (static_cast<size_t>(pl.nctas) + B + dyn_slots) * Hq;
+    pl.bytes = pl.n_part * (kDecD + 1) * sizeof(float) + (static_cast<size_t>(B) + 2) * sizeof(int);
   } else {
     pl.n_part = static_cast<size_t>(B) * pl.nsplit * Hq;
     pl.bytes = pl.n_part * (kDecD + 1) * sizeof(float);
@@ -720,9 +877,13 @@ DecodePlan make_plan(int B, int Hq, int Hkv, int max_pages_per_seq, int nsm) {
   // streamed: one consumer warp per KV head, its G <= 8 query heads as MMA rows
   pl.streamed = Hkv <= kDecWarps && nsm > 0;
   if (pl.streamed) {
-    pl.nctas = nsm;
+    pl.nctas = std::min(nsm, kMaxStreamCtas);
     pl.nstages = kStreamSmemBudget / (2 * stage_kv_bytes(Hkv));
     if (pl.nstages > kMaxStages) pl.nstages = kMaxStages;
+    // enough units for the dynamic tenth of every share of the longest possible list
+    const long long h_max = 2LL * B * max_pages_per_seq;
+    const long long per_cta = ((h_max + pl.nctas - 1) / pl.nctas) / kDynDiv / kDynUnit + 1;
+    pl.dyn_units_cap = static_cast<int>(std::min<long long>(per_cta * pl.nctas, 1 << 24));
   } else {
     pl.pps = direct_pps(B, max_pages_per_seq);
     pl.nsplit = (max_pages_per_seq + pl.pps - 1) / pl.pps;
@@ -735,7 +896,8 @@ template <int G>
 int launch_kernels(const DecodeParams& prm, const DecodePlan& pl, const CUtensorMap& tmK,
                    const CUtensorMap& tmV, cudaStream_t stream, int device) {
   if (pl.streamed) {
-    const int smem = pl.nstages * 2 * stage_kv_bytes(prm.Hkv) + 1024;
+    const int smem = pl.nstages * 2 * stage_kv_bytes(prm.Hkv) + 1024 +
+                     (prm.hb_in_smem ? (prm.B + 1) * 4 : 0);
     {
       // the shared-memory limit is a property of the function on each device
       static bool attr_done[64] = {};
@@ -745,7 +907,7 @@ int launch_kernels(const DecodeParams& prm, const DecodePlan& pl, const CUtensor
       if (!attr_done[device]) {
         cudaError_t e = cudaFuncSetAttribute(fa_decode_stream_kernel<G>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kStreamSmemBudget + 1024);
+                                             kStreamSmemBudget + 1024 + kHbSmemMax * 4);
         if (e != cudaSuccess)
           return set_error(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
         attr_done[device] = true;
@@ -766,8 +928,8 @@ int launch_kernels(const DecodeParams& prm, const DecodePlan& pl, const CUtensor
     cfg.blockDim = dim3(kStreamThreads);
     cfg.dynamicSmemBytes = smem;
     cudaLaunchKernelEx(&cfg, fa_decode_stream_kernel<G>, tmK, tmV, prm);
-    cfg.gridDim = dim3((prm.B * prm.Hq + 3) / 4);
-    cfg.blockDim = dim3(128);
+    cfg.gridDim = dim3(prm.B);
+    cfg.blockDim = dim3(kMergeWarps * 32);
     cfg.dynamicSmemBytes = 0;
     cudaLaunchKernelEx(&cfg, fa_decode_stream_merge_kernel, prm);
   } else {
@@ -801,6 +963,8 @@ int run_decode(const void* q, const void* kcache, const void* vcache, const int3
   prm.nsplit = pl.nsplit;
   prm.nctas = pl.nctas;
   prm.nstages = pl.nstages;
+  prm.dyn_units_cap = pl.dyn_units_cap;
+  prm.hb_in_smem = B + 1 <= kHbSmemMax ? 1 : 0;
   prm.scale_log2 = scale * kLog2e;
   prm.err = device_error_word(device);
   if (!prm.err) return set_error(FA_ERR_CUDA, "device error word unavailable");
@@ -811,6 +975,7 @@ int run_decode(const void* q, const void* kcache, const void* vcache, const int3
   prm.ws_o = static_cast<float*>(ws);
   prm.ws_lse = prm.ws_o + pl.n_part * kDecD;
   prm.hb = reinterpret_cast<int*>(prm.ws_lse + pl.n_part);
+  prm.dyn_next = prm.hb + (B + 1);
   CUtensorMap tmK, tmV;
   if (pl.streamed) {
     // K and V caches viewed as [Hkv][num_pages * 16 tokens][128]: box {64, 8, Hkv}
@@ -923,6 +1088,15 @@ int scratch_address(int device, float** out) {
 // the direct schedule with chunks widened until its partials fit.
 int plan_noalloc(int B, int Hq, int Hkv, int max_pages_per_seq, int nsm, DecodePlan* out) {
   DecodePlan pl = make_plan(B, Hq, Hkv, max_pages_per_seq, nsm);
+  if (pl.streamed && pl.bytes > kNoAllocScratchBytes) {
+    // fewer dynamic units (each then covers more half-pages), or none
+    const long long rows_fit =
+        (static_cast<long long>(kNoAllocScratchBytes) - (static_cast<long long>(B) + 2) * 4) /
+        ((kDecD + 1) * 4) / Hq;
+    const long long cap = rows_fit - pl.nctas - 2LL * B;
+    pl.dyn_units_cap = cap > 0 ? static_cast<int>(std::min<long long>(cap, pl.dyn_units_cap)) : 0;
+    finish_plan(pl, B, Hq, Hkv);
+  }
   if (!pl.streamed) {
     while (pl.bytes > kNoAllocScratchBytes && pl.nsplit > 1) {
       pl.pps *= 2;
