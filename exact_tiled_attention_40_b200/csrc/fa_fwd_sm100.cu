@@ -31,6 +31,7 @@
 // The rescale is lazy: a row's reference maximum only moves when the new tile
 // maximum exceeds it by more than 2^8, so P stays <= 256 and O is rescaled only
 // on those rare tiles.  Exactness is unaffected: O and L share the reference.
+#include <algorithm>
 #include <cfloat>
 #include <cstdio>
 #include <mutex>
@@ -64,7 +65,7 @@ struct FwdLayout {
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
-  static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 4 + 2 + 1;
+  static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 4 + 2 + 1 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + slack for 1024-byte alignment
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -75,6 +76,7 @@ struct FwdParams {
   float* lse;
   int B, Hq, Hkv, Nq, Nk;
   int num_mpairs;
+  int num_items;      // num_mpairs * B * Hq work items, heaviest first
   int causal;
   float scale_log2;   // scale * log2(e)
   int* err;
@@ -90,6 +92,32 @@ __device__ __forceinline__ int kv_tiles_for(int first_row, const FwdParams& p) {
   return min(nk_tiles, max_key / kBN + 1);
 }
 
+// Work item i: (batch, head, pair of 128-row query tiles); with a causal mask the
+// pairs are ordered heaviest first.
+struct FwdItem {
+  int bh, b, hkv, q_row0, n0, n1;
+};
+__device__ __forceinline__ FwdItem item_of(int i, const FwdParams& p) {
+  FwdItem it;
+  const int BH = p.B * p.Hq;
+  const int mrev = i / BH;
+  it.bh = i - mrev * BH;
+  const int mpair = p.causal ? (p.num_mpairs - 1 - mrev) : mrev;
+  it.b = it.bh / p.Hq;
+  it.hkv = (it.bh - it.b * p.Hq) / (p.Hq / p.Hkv);
+  it.q_row0 = mpair * 2 * kBM;
+  it.n0 = kv_tiles_for(it.q_row0, p);
+  it.n1 = kv_tiles_for(it.q_row0 + kBM, p);
+  return it;
+}
+// The r-th item of CTA c: rounds of gridDim items, alternately left to right and
+// right to left (with the heaviest-first order this balances the CTAs' totals
+// about as well as handing items out dynamically); -1 when none is left.
+__device__ __forceinline__ int item_index(int c, int r, int C, int total) {
+  const int i = r * C + ((r & 1) ? C - 1 - c : c);
+  return i < total ? i : -1;
+}
+
 template <int D, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -103,19 +131,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // ---- work item: (batch, head, pair of query tiles); causal: heaviest first
-  const int BH = p.B * p.Hq;
-  const int mrev = blockIdx.x / BH;
-  const int bh = blockIdx.x - mrev * BH;
-  const int mpair = p.causal ? (p.num_mpairs - 1 - mrev) : mrev;
-  const int b = bh / p.Hq;
-  const int h = bh - b * p.Hq;
-  const int hkv = h / (p.Hq / p.Hkv);
-  const int q_row0 = mpair * 2 * kBM;
-  int n_kv[2];
-  n_kv[0] = kv_tiles_for(q_row0, p);
-  n_kv[1] = kv_tiles_for(q_row0 + kBM, p);
-  const int n_max = max(n_kv[0], n_kv[1]);
+  const int C = gridDim.x;
+  const int cta = blockIdx.x;
 
   auto bar = [&](int i) -> uint32_t { return sbase + L::kBarOff + 8 * i; };
   auto q_full = [&](int t) { return bar(t); };
@@ -127,6 +144,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto p_half = [&](int t, int h) { return bar(4 + 2 * L::kSlots + 2 * t + h); };
   auto o_full = [&](int t) { return bar(8 + 2 * L::kSlots + t); };
   const uint32_t mma_done = bar(10 + 2 * L::kSlots);
+  // Q smem may be refilled: every S MMA of the item has read it
+  const uint32_t q_empty = bar(11 + 2 * L::kSlots);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
@@ -143,6 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(kv_empty(s), 1);
     }
     mbar_init(mma_done, 1);
+    mbar_init(q_empty, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -158,52 +178,62 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_dec<kRegsControl>();
     if (warp == 8) {
       // ------------------------------------------------------------ TMA producer
-      if (lane == 0 && n_max > 0) {
+      // Items in order; per item both Q tiles (a tile past Nq reads as zeros),
+      // then K_j, V_j through the ring, whose position runs on across items.
+      if (lane == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
-        for (int t = 0; t < 2; ++t) {
-          if (n_kv[t] == 0) continue;
-          mbar_arrive_expect_tx(q_full(t), L::kTileBytes);
-          const uint32_t dst = sbase + L::kQOff + t * L::kTileBytes;
-          for (int c = 0; c < L::kChunks; ++c)
-            tma_load_3d(dst + c * L::kChunkBytes, &tmQ, q_full(t), c * 64, q_row0 + t * kBM, bh);
-        }
-        const int kv_z = b * p.Hkv + hkv;
-        int issued = 0;
-        for (int j = 0; j < n_max; ++j) {
-          bool ok = true;
-          for (int w = 0; w < 2; ++w) {
-            const int pos = 2 * j + w;
-            const int slot = pos % L::kSlots;
-            const uint32_t ph = (pos / L::kSlots) & 1;
-            if (!mbar_wait(kv_empty(slot), ph ^ 1, abort_flag, p.err, p.timeout_ns)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(kv_full(slot), L::kTileBytes);
-            const uint32_t dst = sbase + L::kKVOff + slot * L::kTileBytes;
-            const void* tm = w ? static_cast<const void*>(&tmV) : static_cast<const void*>(&tmK);
-            for (int c = 0; c < L::kChunks; ++c)
-              tma_load_3d(dst + c * L::kChunkBytes, tm, kv_full(slot), c * 64, j * kBN, kv_z);
-            ++issued;
+        int pos = 0, items = 0;
+        bool ok = true;
+        for (int r = 0; ok; ++r) {
+          const int i = item_index(cta, r, C, p.num_items);
+          if (i < 0) break;
+          const FwdItem it = item_of(i, p);
+          const int n_max = max(it.n0, it.n1);
+          if (n_max == 0) continue;
+          if (items > 0 && !mbar_wait(q_empty, (items - 1) & 1, abort_flag, p.err, p.timeout_ns))
+            break;
+          for (int t = 0; t < 2; ++t) {
+            mbar_arrive_expect_tx(q_full(t), L::kTileBytes);
+            const uint32_t dst = sbase + L::kQOff + t * L::kTileBytes;
+            for (int ch = 0; ch < L::kChunks; ++ch)
+              tma_load_3d(dst + ch * L::kChunkBytes, &tmQ, q_full(t), ch * 64,
+                          it.q_row0 + t * kBM, it.bh);
           }
-          if (!ok) break;
+          ++items;
+          const int kv_z = it.b * p.Hkv + it.hkv;
+          for (int j = 0; j < n_max && ok; ++j) {
+            for (int w = 0; w < 2; ++w, ++pos) {
+              const int slot = pos % L::kSlots;
+              const uint32_t ph = (pos / L::kSlots) & 1;
+              if (!mbar_wait(kv_empty(slot), ph ^ 1, abort_flag, p.err, p.timeout_ns)) {
+                ok = false;
+                break;
+              }
+              mbar_arrive_expect_tx(kv_full(slot), L::kTileBytes);
+              const uint32_t dst = sbase + L::kKVOff + slot * L::kTileBytes;
+              const void* tm = w ? static_cast<const void*>(&tmV) : static_cast<const void*>(&tmK);
+              for (int ch = 0; ch < L::kChunks; ++ch)
+                tma_load_3d(dst + ch * L::kChunkBytes, tm, kv_full(slot), ch * 64, j * kBN, kv_z);
+            }
+          }
         }
         // Every issued copy must land before the CTA may exit (also on abort).
         volatile int no_abort = 0;
-        for (int t = 0; t < 2; ++t)
-          if (n_kv[t] > 0) mbar_wait(q_full(t), 0, &no_abort, p.err, p.timeout_ns);
-        for (int s = 0; s < L::kSlots && s < issued; ++s) {
-          const int last = s + ((issued - 1 - s) / L::kSlots) * L::kSlots;
-          mbar_wait(kv_full(s), (last / L::kSlots) & 1, &no_abort, p.err, p.timeout_ns);
+        if (items > 0)
+          for (int t = 0; t < 2; ++t)
+            mbar_wait(q_full(t), (items - 1) & 1, &no_abort, p.err, p.timeout_ns);
+        for (int sl = 0; sl < L::kSlots && sl < pos; ++sl) {
+          const int last = sl + ((pos - 1 - sl) / L::kSlots) * L::kSlots;
+          mbar_wait(kv_full(sl), (last / L::kSlots) & 1, &no_abort, p.err, p.timeout_ns);
         }
       }
     } else if (warp == 9) {
       // ------------------------------------------------------------ MMA issuer
       // The whole warp runs the waits, loop counters and descriptor arithmetic
       // (all warp-uniform); one elected lane issues the MMAs and commits.
-      if (n_max > 0) {
+      {
         const bool leader = elect_one();
         constexpr uint32_t idesc_s = idesc_f16(kBM, kBN, BF16, false);
         constexpr uint32_t idesc_pv = idesc_f16(kBM, D, BF16, true);
@@ -252,47 +282,63 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         };
         bool ok = true;
-        if (n_kv[0] > 0) ok = wait(q_full(0), 0);
-        if (ok && n_kv[1] > 0) ok = wait(q_full(1), 0);
-        if (ok) ok = wait(kv_full(slot_of(0)), phase_of(0));
-        if (ok) {
-          tc_fence_after();
-          if (n_kv[0] > 0) issue_s(0, slot_of(0));
-          if (n_kv[1] > 0) issue_s(1, slot_of(0));
-          commit(kv_empty(slot_of(0)));
-        }
-        for (int j = 0; j < n_max && ok; ++j) {
-          const int vpos = 2 * j + 1;
-          const int kpos = 2 * j + 2;
-          const bool has_next = j + 1 < n_max;
-          ok = wait(kv_full(slot_of(vpos)), phase_of(vpos));
-          bool k_ready = false;   // K_{j+1} is waited for just before its first use
-  #pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            if (!ok || j >= (t ? n_kv[1] : n_kv[0])) continue;
-            ok = wait(p_half(t, 0), j & 1);
-            if (!ok) continue;
-            tc_fence_after();
-            issue_pv_half(t, slot_of(vpos), 0, j > 0);
-            ok = wait(p_half(t, 1), j & 1);
-            if (!ok) continue;
-            tc_fence_after();
-            issue_pv_half(t, slot_of(vpos), 1, true);
-            if (j + 1 < (t ? n_kv[1] : n_kv[0])) {
-              if (!k_ready) {
-                ok = wait(kv_full(slot_of(kpos)), phase_of(kpos));
-                k_ready = true;
-                if (!ok) continue;
-                tc_fence_after();
-              }
-              issue_s(t, slot_of(kpos));
-            } else {
-              commit(o_full(t));
-            }
-          }
+        int pos = 0, items = 0;
+        int tiles[2] = {0, 0};   // S tiles of each query-tile slot in earlier items (phases)
+        for (int r = 0; ok; ++r) {
+          const int i = item_index(cta, r, C, p.num_items);
+          if (i < 0) break;
+          const FwdItem it = item_of(i, p);
+          const int n_max = max(it.n0, it.n1);
+          if (n_max == 0) continue;
+          ok = wait(q_full(0), items & 1);
+          if (ok) ok = wait(q_full(1), items & 1);
+          if (ok) ok = wait(kv_full(slot_of(pos)), phase_of(pos));
           if (!ok) break;
-          commit(kv_empty(slot_of(vpos)));
-          if (has_next) commit(kv_empty(slot_of(kpos)));
+          ++items;
+          tc_fence_after();
+          if (it.n0 > 0) issue_s(0, slot_of(pos));
+          if (it.n1 > 0) issue_s(1, slot_of(pos));
+          commit(kv_empty(slot_of(pos)));
+          if (n_max == 1) commit(q_empty);
+          for (int j = 0; j < n_max && ok; ++j) {
+            const int vpos = pos + 2 * j + 1;
+            const int kpos = pos + 2 * j + 2;
+            const bool has_next = j + 1 < n_max;
+            ok = wait(kv_full(slot_of(vpos)), phase_of(vpos));
+            bool k_ready = false;   // K_{j+1} is waited for just before its first use
+  #pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              const int nt = t ? it.n1 : it.n0;
+              if (!ok || j >= nt) continue;
+              const uint32_t par = static_cast<uint32_t>((tiles[t] + j) & 1);
+              ok = wait(p_half(t, 0), par);
+              if (!ok) continue;
+              tc_fence_after();
+              issue_pv_half(t, slot_of(vpos), 0, j > 0);
+              ok = wait(p_half(t, 1), par);
+              if (!ok) continue;
+              tc_fence_after();
+              issue_pv_half(t, slot_of(vpos), 1, true);
+              if (j + 1 < nt) {
+                if (!k_ready) {
+                  ok = wait(kv_full(slot_of(kpos)), phase_of(kpos));
+                  k_ready = true;
+                  if (!ok) continue;
+                  tc_fence_after();
+                }
+                issue_s(t, slot_of(kpos));
+              } else {
+                commit(o_full(t));
+              }
+            }
+            if (!ok) break;
+            if (j + 2 == n_max) commit(q_empty);   // the item's last S MMAs are issued
+            commit(kv_empty(slot_of(vpos)));
+            if (has_next) commit(kv_empty(slot_of(kpos)));
+          }
+          pos += 2 * n_max;
+          tiles[0] += it.n0;
+          tiles[1] += it.n1;
         }
         // All issued MMAs must complete before TMEM is released (also on abort).
         commit(mma_done);
@@ -305,18 +351,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ softmax warpgroups
     const int t = warp >> 2;
     const int r = tid & 127;
-    const int row = q_row0 + t * kBM + r;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + t * 128;
     const uint32_t tO = tmem + lane_base + 256 + t * D;
-    const int n = t ? n_kv[1] : n_kv[0];
-    const size_t row_index = static_cast<size_t>(bh) * p.Nq + row;
+    int tiles = 0, outs = 0;     // S tiles and O tiles of this slot in earlier items (phases)
+    bool ok = true;
+    for (int ri = 0; ok; ++ri) {
+    const int item = item_index(cta, ri, C, p.num_items);
+    if (item < 0) break;
+    const FwdItem it = item_of(item, p);
+    const int q_row0 = it.q_row0;
+    const int row = q_row0 + t * kBM + r;
+    const int n = t ? it.n1 : it.n0;
+    const size_t row_index = static_cast<size_t>(it.bh) * p.Nq + row;
     using Out = uint16_t;
     Out* o_row = reinterpret_cast<Out*>(p.o) + row_index * D;
     if (n == 0) {
-      if (row < p.Nq && q_row0 + t * kBM < p.Nq) {   // only reached when Nk == 0
+      if (max(it.n0, it.n1) == 0 && row < p.Nq) {   // only reached when Nk == 0
         uint4 z = make_uint4(0, 0, 0, 0);
-        for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(o_row)[c] = z;
+        for (int ch = 0; ch < D / 8; ++ch) reinterpret_cast<uint4*>(o_row)[ch] = z;
         if (p.lse) p.lse[row_index] = -INFINITY;
       }
     } else {
@@ -324,11 +377,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       float l = 0.f;
       const int off = p.Nk - p.Nq;
       const int tile_first = q_row0 + t * kBM;
-      bool ok = true;
       for (int j = 0; j < n; ++j) {
         // tcgen05.ld/st/wait are warp-collective: every branch around them is
         // made warp-uniform, also on the abort path.
-        const bool got = mbar_wait(s_full(t), j & 1, abort_flag, p.err, p.timeout_ns);
+        const bool got = mbar_wait(s_full(t), (tiles + j) & 1, abort_flag, p.err, p.timeout_ns);
         if (!__all_sync(0xffffffffu, got)) {
           ok = false;
           break;
@@ -444,8 +496,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(p_half(t, 1));
       }
-      const bool fin = ok && mbar_wait(o_full(t), 0, abort_flag, p.err, p.timeout_ns);
-      if (__all_sync(0xffffffffu, fin)) {
+      tiles += n;
+      const bool fin = ok && mbar_wait(o_full(t), outs & 1, abort_flag, p.err, p.timeout_ns);
+      ++outs;
+      if (!__all_sync(0xffffffffu, fin)) {
+        ok = false;
+      } else {
         tc_fence_after();
         const float inv_l = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
@@ -471,6 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           p.lse[row_index] = l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
       }
     }
+    }
   }
 
   tc_fence_before();
@@ -492,6 +549,19 @@ int encode_3d(CUtensorMap* m, const void* base, bool bf16, int D, int N, int Z) 
                                static_cast<uint64_t>(N) * static_cast<uint64_t>(D) * 2};
   const uint32_t box[3] = {64, 128, 1};
   return encode_tensor_map_16bit(m, base, bf16, 3, dims, strides, box);
+}
+
+int fwd_sm_count(int device) {
+  static int cached[64] = {};
+  static std::mutex mu;
+  std::lock_guard<std::mutex> g(mu);
+  if (device < 0 || device >= 64) return 0;
+  if (!cached[device]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) n = 0;
+    cached[device] = n;
+  }
+  return cached[device];
 }
 
 template <int D, bool BF16>
@@ -537,8 +607,14 @@ int launch_typed(const void* q, const void* k, const void* v, void* o, float* ls
   prm.err = device_error_word(device);
   prm.timeout_ns = kWaitLimitNs;
   if (!prm.err) return set_error(FA_ERR_CUDA, "device error word unavailable");
-  const long long grid = static_cast<long long>(prm.num_mpairs) * B * Hq;
-  if (grid > 0x7fffffffLL) return set_error(FA_ERR_UNSUPPORTED, "grid too large");
+  const long long items = static_cast<long long>(prm.num_mpairs) * B * Hq;
+  if (items > 0x7fffffffLL) return set_error(FA_ERR_UNSUPPORTED, "too many work items");
+  prm.num_items = static_cast<int>(items);
+  // persistent: one CTA per SM (at most one per item), each walking its items
+  const int nsm = fwd_sm_count(device);
+  if (nsm <= 0) return set_error(FA_ERR_CUDA, "cannot read the SM count of device %d", device);
+  const int grid = static_cast<int>(std::min<long long>(items, nsm));
+  if (grid == 0) return FA_OK;
   fa_fwd_kernel<D, BF16><<<static_cast<unsigned>(grid), kThreads, L::kSmemBytes, stream>>>(
       tq, tk, tv, prm);
   cudaError_t e = cudaGetLastError();
