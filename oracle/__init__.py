@@ -13,4 +13,5 @@ from .attention_fp64 import (  # noqa: F401
     kv_head_of,
     merge_partials,
     softmax_rows,
+    varlen_attention,
 )

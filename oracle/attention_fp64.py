@@ -283,3 +283,43 @@ def decode_paged(q, kcache, vcache, block_table, seq_lens, scale: float, page_si
         O[b] = o[0, :, 0, :]
         LSE[b] = lse[0, :, 0]
     return O, LSE
+
+
+def varlen_attention(q, k, v, cu_seqlens_q, cu_seqlens_k, scale: float, causal: bool):
+    """Attention over a ragged batch packed without padding.
+
+    [devh] example 3 combines the causal rule with a padding mask, and [cabseo]
+    "Continuous batching" groups sequences of different lengths in one batch.
+    Reading: a packed batch of B sequences is the padded batch with a key
+    padding mask, where sequence b's queries see only sequence b's keys.
+    Sequence b owns query rows [cu_seqlens_q[b], cu_seqlens_q[b+1]) and key rows
+    [cu_seqlens_k[b], cu_seqlens_k[b+1]); the definition ``attention`` is
+    applied to each sequence on its own (causal: bottom-right aligned within the
+    sequence).
+
+    q [total_q, Hq, D]; k, v [total_k, Hkv, D]; cu_seqlens_* int [B + 1].
+    Returns O [total_q, Hq, D] and LSE [Hq, total_q] (natural log).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    cq = np.asarray(cu_seqlens_q, dtype=np.int64)
+    ck = np.asarray(cu_seqlens_k, dtype=np.int64)
+    if cq.shape != ck.shape or cq.ndim != 1 or cq[0] != 0 or ck[0] != 0:
+        raise ValueError("cu_seqlens must be [B + 1] offsets starting at 0")
+    if np.any(np.diff(cq) < 0) or np.any(np.diff(ck) < 0):
+        raise ValueError("cu_seqlens must be non-decreasing")
+    total_q, Hq, D = q.shape
+    O = np.zeros((total_q, Hq, D))
+    LSE = np.full((Hq, total_q), -np.inf)
+    for b in range(len(cq) - 1):
+        q0, q1, k0, k1 = cq[b], cq[b + 1], ck[b], ck[b + 1]
+        if q1 == q0:
+            continue
+        qb = np.transpose(q[q0:q1], (1, 0, 2))[None]      # [1, Hq, Nq_b, D]
+        kb = np.transpose(k[k0:k1], (1, 0, 2))[None]      # [1, Hkv, Nk_b, D]
+        vb = np.transpose(v[k0:k1], (1, 0, 2))[None]
+        o, lse = attention(qb, kb, vb, scale, causal)
+        O[q0:q1] = np.transpose(o[0], (1, 0, 2))
+        LSE[:, q0:q1] = lse[0]
+    return O, LSE

@@ -264,3 +264,93 @@ def test_pins_catch_missing_normalisation(monkeypatch):
     monkeypatch.setattr(oracle_mod, "softmax_rows", unnormalised)
     O_bad, _ = oracle_mod.attention(q, k, v, case["scale"], case["causal"])
     assert np.max(np.abs(O_bad - np.array(case["O"]))) > 1e-3
+
+
+# ---------------------------------------------------------------- ragged batches
+def _packed_case(Nq, Nk, Hq, Hkv, D, seed):
+    cu_q = np.concatenate([[0], np.cumsum(Nq)]).astype(np.int64)
+    cu_k = np.concatenate([[0], np.cumsum(Nk)]).astype(np.int64)
+    q = rand((int(cu_q[-1]), Hq, D), seed)
+    k = rand((int(cu_k[-1]), Hkv, D), seed + 1)
+    v = rand((int(cu_k[-1]), Hkv, D), seed + 2)
+    return q, k, v, cu_q, cu_k
+
+
+def _padded_library(q, k, v, cu_q, cu_k, scale, causal):
+    """The padded-batch formulation of a ragged batch, through torch's float64
+    scaled_dot_product_attention with an explicit per-sequence boolean mask:
+    key j of sequence b is visible to its query i iff j < Nk_b (and, causal,
+    j <= i + Nk_b - Nq_b).  Returns O and LSE in the packed layouts; rows with no
+    visible key are NaN."""
+    B = len(cu_q) - 1
+    Nq = np.diff(cu_q)
+    Nk = np.diff(cu_k)
+    Mq, Mk = max(1, int(Nq.max())), max(1, int(Nk.max()))
+    Hq, D = q.shape[1], q.shape[2]
+    Hkv = k.shape[1]
+    qp = np.zeros((B, Hq, Mq, D))
+    kp = np.zeros((B, Hkv, Mk, D))
+    vp = np.zeros((B, Hkv, Mk, D))
+    mask = np.zeros((B, 1, Mq, Mk), dtype=bool)
+    for b in range(B):
+        qp[b, :, :Nq[b]] = np.transpose(q[cu_q[b]:cu_q[b + 1]], (1, 0, 2))
+        kp[b, :, :Nk[b]] = np.transpose(k[cu_k[b]:cu_k[b + 1]], (1, 0, 2))
+        vp[b, :, :Nk[b]] = np.transpose(v[cu_k[b]:cu_k[b + 1]], (1, 0, 2))
+        i = np.arange(Mq)[:, None]
+        j = np.arange(Mk)[None, :]
+        ok = j < Nk[b]
+        if causal:
+            ok = ok & (j <= i + Nk[b] - Nq[b])
+        mask[b, 0] = ok
+    tq, tk, tv = (torch.from_numpy(x) for x in (qp, kp, vp))
+    rep = Hq // Hkv
+    tk = tk.repeat_interleave(rep, dim=1)
+    tv = tv.repeat_interleave(rep, dim=1)
+    tm = torch.from_numpy(mask)
+    o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=tm, scale=scale)
+    s = (scale * (tq @ tk.transpose(-1, -2))).masked_fill(~tm, float("-inf"))
+    lse = torch.logsumexp(s, dim=-1)
+    O = np.zeros(q.shape)
+    L = np.zeros((Hq, q.shape[0]))
+    for b in range(B):
+        O[cu_q[b]:cu_q[b + 1]] = np.transpose(o[b, :, :Nq[b]].numpy(), (1, 0, 2))
+        L[:, cu_q[b]:cu_q[b + 1]] = lse[b, :, :Nq[b]].numpy()
+    return O, L
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_matches_padded_library_attention(causal):
+    Nq = np.array([5, 0, 9, 1, 3])
+    Nk = np.array([7, 3, 9, 4, 3])
+    q, k, v, cu_q, cu_k = _packed_case(Nq, Nk, 4, 2, 8, 60)
+    O, L = oracle.varlen_attention(q, k, v, cu_q, cu_k, 0.4, causal)
+    O_ref, L_ref = _padded_library(q, k, v, cu_q, cu_k, 0.4, causal)
+    np.testing.assert_allclose(O, O_ref, atol=TIGHT)
+    np.testing.assert_allclose(L, L_ref, atol=TIGHT)
+
+
+def test_varlen_sequences_without_keys_and_independence():
+    Nq = np.array([4, 3, 5])
+    Nk = np.array([6, 0, 5])
+    q, k, v, cu_q, cu_k = _packed_case(Nq, Nk, 2, 1, 4, 70)
+    O, L = oracle.varlen_attention(q, k, v, cu_q, cu_k, 0.5, False)
+    assert np.all(O[4:7] == 0) and np.all(L[:, 4:7] == -np.inf)       # sequence 1: no keys
+    # changing sequence 2's keys and values leaves sequence 0 untouched
+    k2, v2 = k.copy(), v.copy()
+    k2[6:] += 1.0
+    v2[6:] -= 2.0
+    O2, L2 = oracle.varlen_attention(q, k2, v2, cu_q, cu_k, 0.5, False)
+    assert np.array_equal(O2[:4], O[:4]) and np.array_equal(L2[:, :4], L[:, :4])
+    assert np.max(np.abs(O2[7:] - O[7:])) > 1e-3
+
+
+def test_pins_catch_a_varlen_offset_mixup():
+    """Using the query offsets for the keys (a plausible slip) fails the padded check."""
+    Nq = np.array([3, 6, 2])
+    Nk = np.array([8, 6, 5])
+    q, k, v, cu_q, cu_k = _packed_case(Nq, Nk, 2, 2, 4, 80)
+    O_ref, _ = _padded_library(q, k, v, cu_q, cu_k, 0.5, True)
+    cu_bad = cu_k.copy()
+    cu_bad[1:-1] = cu_q[1:-1]                 # keys split at the query boundaries
+    O_bad, _ = oracle.varlen_attention(q, k, v, cu_q, cu_bad, 0.5, False)
+    assert np.max(np.abs(O_bad - O_ref)) > 1e-3
