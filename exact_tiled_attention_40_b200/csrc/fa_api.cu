@@ -137,7 +137,36 @@ int fwd_common(const void* q, const void* k, const void* v, void* o, float* lse,
   if (B == 0 || Hq == 0 || Nq == 0) return FA_OK;
   int dev;
   if ((rc = current_sm100(&dev)) != FA_OK) return rc;
-  return launch_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal, bf16, stream, dev);
+  return launch_fwd(q, k, v, o, lse, nullptr, nullptr, 0, 0, B, Hq, Hkv, Nq, Nk, D, scale, causal,
+                    bf16, stream, dev);
+}
+
+int varlen_common(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int32_t* cu_q, const int32_t* cu_k, int B, int Hq, int Hkv,
+                  int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int D, float scale,
+                  int causal, cudaStream_t stream, bool bf16) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || max_seqlen_q < 0 || max_seqlen_k < 0 || total_q < 0 ||
+      total_k < 0)
+    return set_error(FA_ERR_INVALID_ARG, "negative size");
+  if (!(std::isfinite(scale) && scale > 0.f))
+    return set_error(FA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (D != 64 && D != 128)
+    return set_error(FA_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", D);
+  if (B == 0 || Hq == 0 || total_q == 0 || max_seqlen_q == 0) return FA_OK;
+  if (Hkv <= 0 || Hq % Hkv != 0)
+    return set_error(FA_ERR_INVALID_ARG, "Hq (%d) must be a positive multiple of Hkv (%d)", Hq,
+                     Hkv);
+  if (!q || !o || !cu_q || !cu_k || (total_k > 0 && (!k || !v)))
+    return set_error(FA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(o) || (total_k > 0 && (!aligned16(k) || !aligned16(v))))
+    return set_error(FA_ERR_INVALID_ARG, "q, k, v and o must be 16-byte aligned");
+  if (static_cast<long long>(total_q) * Hq > 0x7fffffffLL ||
+      static_cast<long long>(max_seqlen_q) + 256 > 0x7fffffffLL)
+    return set_error(FA_ERR_INVALID_ARG, "total_q * Hq too large");
+  int dev, rc;
+  if ((rc = current_sm100(&dev)) != FA_OK) return rc;
+  return launch_fwd(q, k, v, o, lse, cu_q, cu_k, total_q, total_k, B, Hq, Hkv, max_seqlen_q,
+                    max_seqlen_k, D, scale, causal, bf16, stream, dev);
 }
 
 }  // namespace
@@ -155,6 +184,24 @@ int fa_fwd_fp16(const void* q, const void* k, const void* v, void* o, float* lse
                 int Hkv, int Nq, int Nk, int D, float scale, int causal, fa_stream_t stream) {
   return fa::fwd_common(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal,
                         reinterpret_cast<cudaStream_t>(stream), false);
+}
+
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B, int Hq,
+                  int Hkv, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int D,
+                  float scale, int causal, fa_stream_t stream) {
+  return fa::varlen_common(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, Hq, Hkv, max_seqlen_q,
+                           max_seqlen_k, total_q, total_k, D, scale, causal,
+                           reinterpret_cast<cudaStream_t>(stream), true);
+}
+
+int fa_fwd_varlen_fp16(const void* q, const void* k, const void* v, void* o, float* lse,
+                       const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B, int Hq,
+                       int Hkv, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+                       int D, float scale, int causal, fa_stream_t stream) {
+  return fa::varlen_common(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, Hq, Hkv, max_seqlen_q,
+                           max_seqlen_k, total_q, total_k, D, scale, causal,
+                           reinterpret_cast<cudaStream_t>(stream), false);
 }
 
 int fa_decode_paged(const void* q, const void* kcache, const void* vcache,

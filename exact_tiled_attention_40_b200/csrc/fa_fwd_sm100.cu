@@ -74,6 +74,13 @@ struct FwdLayout {
 struct FwdParams {
   void* o;
   float* lse;
+  // Ragged batch packed without padding (null: the dense [B, H, N, D] layout):
+  // sequence b owns query rows [cu_q[b], cu_q[b+1]) of q/o [total_q, Hq, D] and
+  // key rows [cu_k[b], cu_k[b+1]) of k/v [total_k, Hkv, D]; lse is [Hq, total_q].
+  // Nq, Nk then bound the sequence lengths.
+  const int* cu_q;
+  const int* cu_k;
+  int total_q, total_k;
   int B, Hq, Hkv, Nq, Nk;
   int num_mpairs;
   int num_items;      // num_mpairs * B * Hq work items, heaviest first
@@ -83,19 +90,23 @@ struct FwdParams {
   uint64_t timeout_ns;
 };
 
-__device__ __forceinline__ int kv_tiles_for(int first_row, const FwdParams& p) {
-  if (first_row >= p.Nq) return 0;
-  const int nk_tiles = (p.Nk + kBN - 1) / kBN;
-  if (!p.causal) return nk_tiles;
-  const int last_row = min(first_row + kBM - 1, p.Nq - 1);
-  const int max_key = last_row + (p.Nk - p.Nq);
+// Key tiles needed by the query tile starting at first_row of a sequence with Nq
+// queries and Nk keys.
+__device__ __forceinline__ int kv_tiles_for(int first_row, int Nq, int Nk, int causal) {
+  if (first_row >= Nq) return 0;
+  const int nk_tiles = (Nk + kBN - 1) / kBN;
+  if (!causal) return nk_tiles;
+  const int last_row = min(first_row + kBM - 1, Nq - 1);
+  const int max_key = last_row + (Nk - Nq);
   return min(nk_tiles, max_key / kBN + 1);
 }
 
 // Work item i: (batch, head, pair of 128-row query tiles); with a causal mask the
 // pairs are ordered heaviest first.
 struct FwdItem {
-  int bh, b, hkv, q_row0, n0, n1;
+  int bh, b, h, hkv, q_row0, n0, n1;
+  int q_start, k_start, nq, nk;   // the sequence's rows (dense: 0, 0, Nq, Nk)
+  bool bad;                       // ragged offsets out of range: the item is skipped
 };
 __device__ __forceinline__ FwdItem item_of(int i, const FwdParams& p) {
   FwdItem it;
@@ -104,10 +115,27 @@ __device__ __forceinline__ FwdItem item_of(int i, const FwdParams& p) {
   it.bh = i - mrev * BH;
   const int mpair = p.causal ? (p.num_mpairs - 1 - mrev) : mrev;
   it.b = it.bh / p.Hq;
-  it.hkv = (it.bh - it.b * p.Hq) / (p.Hq / p.Hkv);
+  it.h = it.bh - it.b * p.Hq;
+  it.hkv = it.h / (p.Hq / p.Hkv);
   it.q_row0 = mpair * 2 * kBM;
-  it.n0 = kv_tiles_for(it.q_row0, p);
-  it.n1 = kv_tiles_for(it.q_row0 + kBM, p);
+  it.bad = false;
+  if (p.cu_q) {
+    const int q0 = p.cu_q[it.b], q1 = p.cu_q[it.b + 1];
+    const int k0 = p.cu_k[it.b], k1 = p.cu_k[it.b + 1];
+    it.bad = q0 < 0 || q1 < q0 || q1 > p.total_q || q1 - q0 > p.Nq || k0 < 0 || k1 < k0 ||
+             k1 > p.total_k || (p.causal && q1 - q0 > k1 - k0);
+    it.q_start = q0;
+    it.k_start = k0;
+    it.nq = it.bad ? 0 : q1 - q0;
+    it.nk = it.bad ? 0 : k1 - k0;
+  } else {
+    it.q_start = 0;
+    it.k_start = 0;
+    it.nq = p.Nq;
+    it.nk = p.Nk;
+  }
+  it.n0 = kv_tiles_for(it.q_row0, it.nq, it.nk, p.causal);
+  it.n1 = kv_tiles_for(it.q_row0 + kBM, it.nq, it.nk, p.causal);
   return it;
 }
 // The r-th item of CTA c: rounds of gridDim items, alternately left to right and
@@ -197,9 +225,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int t = 0; t < 2; ++t) {
             mbar_arrive_expect_tx(q_full(t), L::kTileBytes);
             const uint32_t dst = sbase + L::kQOff + t * L::kTileBytes;
-            for (int ch = 0; ch < L::kChunks; ++ch)
-              tma_load_3d(dst + ch * L::kChunkBytes, &tmQ, q_full(t), ch * 64,
-                          it.q_row0 + t * kBM, it.bh);
+            for (int ch = 0; ch < L::kChunks; ++ch) {
+              if (p.cu_q)   // [total_q, Hq, D]: box {64, 1 head, 128 rows}
+                tma_load_3d(dst + ch * L::kChunkBytes, &tmQ, q_full(t), ch * 64, it.h,
+                            it.q_start + it.q_row0 + t * kBM);
+              else          // [B * Hq, Nq, D]: box {64, 128 rows, 1}
+                tma_load_3d(dst + ch * L::kChunkBytes, &tmQ, q_full(t), ch * 64,
+                            it.q_row0 + t * kBM, it.bh);
+            }
           }
           ++items;
           const int kv_z = it.b * p.Hkv + it.hkv;
@@ -214,8 +247,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               mbar_arrive_expect_tx(kv_full(slot), L::kTileBytes);
               const uint32_t dst = sbase + L::kKVOff + slot * L::kTileBytes;
               const void* tm = w ? static_cast<const void*>(&tmV) : static_cast<const void*>(&tmK);
-              for (int ch = 0; ch < L::kChunks; ++ch)
-                tma_load_3d(dst + ch * L::kChunkBytes, tm, kv_full(slot), ch * 64, j * kBN, kv_z);
+              for (int ch = 0; ch < L::kChunks; ++ch) {
+                if (p.cu_q)
+                  tma_load_3d(dst + ch * L::kChunkBytes, tm, kv_full(slot), ch * 64, it.hkv,
+                              it.k_start + j * kBN);
+                else
+                  tma_load_3d(dst + ch * L::kChunkBytes, tm, kv_full(slot), ch * 64, j * kBN,
+                              kv_z);
+              }
             }
           }
         }
@@ -361,13 +400,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (item < 0) break;
     const FwdItem it = item_of(item, p);
     const int q_row0 = it.q_row0;
-    const int row = q_row0 + t * kBM + r;
+    const int row = q_row0 + t * kBM + r;          // within the sequence
     const int n = t ? it.n1 : it.n0;
-    const size_t row_index = static_cast<size_t>(it.bh) * p.Nq + row;
+    if (it.bad && t == 0 && r == 0 && q_row0 == 0) atomicOr(p.err, kErrBadIndex);
+    // o element offset / D and lse offset of this row
+    const size_t o_index = p.cu_q
+        ? static_cast<size_t>(it.q_start + row) * p.Hq + it.h
+        : static_cast<size_t>(it.bh) * p.Nq + row;
+    const size_t row_index = p.cu_q
+        ? static_cast<size_t>(it.h) * p.total_q + it.q_start + row
+        : o_index;
     using Out = uint16_t;
-    Out* o_row = reinterpret_cast<Out*>(p.o) + row_index * D;
+    Out* o_row = reinterpret_cast<Out*>(p.o) + o_index * D;
     if (n == 0) {
-      if (max(it.n0, it.n1) == 0 && row < p.Nq) {   // only reached when Nk == 0
+      if (max(it.n0, it.n1) == 0 && row < it.nq) {   // only reached when Nk == 0
         uint4 z = make_uint4(0, 0, 0, 0);
         for (int ch = 0; ch < D / 8; ++ch) reinterpret_cast<uint4*>(o_row)[ch] = z;
         if (p.lse) p.lse[row_index] = -INFINITY;
@@ -375,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
       float m_used = -INFINITY;
       float l = 0.f;
-      const int off = p.Nk - p.Nq;
+      const int off = it.nk - it.nq;
       const int tile_first = q_row0 + t * kBM;
       for (int j = 0; j < n; ++j) {
         // tcgen05.ld/st/wait are warp-collective: every branch around them is
@@ -394,9 +440,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         const int kbase = j * kBN;
         const bool need_mask =
-            (kbase + kBN > p.Nk) || (p.causal && kbase + kBN - 1 > tile_first + off);
+            (kbase + kBN > it.nk) || (p.causal && kbase + kBN - 1 > tile_first + off);
         if (need_mask) {
-          int lim = p.Nk - 1 - kbase;                       // last visible column
+          int lim = it.nk - 1 - kbase;                      // last visible column
           if (p.causal) lim = min(lim, row + off - kbase);
 #pragma unroll
           for (int e = 0; e < 128; ++e)
@@ -516,14 +562,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float bb = __uint_as_float(ov[2 * e + 1]) * inv_l;
             pk[e] = BF16 ? pack_bf16x2(a, bb) : pack_f16x2(a, bb);
           }
-          if (row < p.Nq) {
+          if (row < it.nq) {
             uint4* dst = reinterpret_cast<uint4*>(o_row + 32 * c);
 #pragma unroll
             for (int v = 0; v < 4; ++v)
               dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
           }
         }
-        if (p.lse && row < p.Nq)
+        if (p.lse && row < it.nq)
           p.lse[row_index] = l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
       }
     }
@@ -550,6 +596,16 @@ int encode_3d(CUtensorMap* m, const void* base, bool bf16, int D, int N, int Z) 
   const uint32_t box[3] = {64, 128, 1};
   return encode_tensor_map_16bit(m, base, bf16, 3, dims, strides, box);
 }
+// 3-D map over a packed [T, H, D] tensor (token-major) with a 64 x 1 x 128 box:
+// the same 128 rows of 128 bytes in shared memory as encode_3d's box.
+int encode_packed(CUtensorMap* m, const void* base, bool bf16, int D, int H, int T) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(H),
+                            static_cast<uint64_t>(T)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2,
+                               static_cast<uint64_t>(H) * static_cast<uint64_t>(D) * 2};
+  const uint32_t box[3] = {64, 1, 128};
+  return encode_tensor_map_16bit(m, base, bf16, 3, dims, strides, box);
+}
 
 int fwd_sm_count(int device) {
   static int cached[64] = {};
@@ -565,7 +621,8 @@ int fwd_sm_count(int device) {
 }
 
 template <int D, bool BF16>
-int launch_typed(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+int launch_typed(const void* q, const void* k, const void* v, void* o, float* lse,
+                 const int* cu_q, const int* cu_k, int total_q, int total_k, int B, int Hq,
                  int Hkv, int Nq, int Nk, float scale, int causal, cudaStream_t stream,
                  int device) {
   using L = FwdLayout<D>;
@@ -585,8 +642,15 @@ int launch_typed(const void* q, const void* k, const void* v, void* o, float* ls
   }
   CUtensorMap tq, tk, tv;
   int rc;
-  if ((rc = encode_3d(&tq, q, BF16, D, Nq, B * Hq)) != FA_OK) return rc;
-  if (Nk > 0) {
+  if (cu_q) {
+    if ((rc = encode_packed(&tq, q, BF16, D, Hq, total_q)) != FA_OK) return rc;
+  } else if ((rc = encode_3d(&tq, q, BF16, D, Nq, B * Hq)) != FA_OK) {
+    return rc;
+  }
+  if (cu_q && total_k > 0) {
+    if ((rc = encode_packed(&tk, k, BF16, D, Hkv, total_k)) != FA_OK) return rc;
+    if ((rc = encode_packed(&tv, v, BF16, D, Hkv, total_k)) != FA_OK) return rc;
+  } else if (!cu_q && Nk > 0) {
     if ((rc = encode_3d(&tk, k, BF16, D, Nk, B * Hkv)) != FA_OK) return rc;
     if ((rc = encode_3d(&tv, v, BF16, D, Nk, B * Hkv)) != FA_OK) return rc;
   } else {
@@ -596,6 +660,10 @@ int launch_typed(const void* q, const void* k, const void* v, void* o, float* ls
   FwdParams prm;
   prm.o = o;
   prm.lse = lse;
+  prm.cu_q = cu_q;
+  prm.cu_k = cu_k;
+  prm.total_q = total_q;
+  prm.total_k = total_k;
   prm.B = B;
   prm.Hq = Hq;
   prm.Hkv = Hkv;
@@ -624,20 +692,18 @@ int launch_typed(const void* q, const void* k, const void* v, void* o, float* ls
 
 }  // namespace
 
-int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+               const int* cu_q, const int* cu_k, int total_q, int total_k, int B, int Hq,
                int Hkv, int Nq, int Nk, int D, float scale, int causal, bool bf16,
                cudaStream_t stream, int device) {
+#define FA_FWD_ARGS q, k, v, o, lse, cu_q, cu_k, total_q, total_k, B, Hq, Hkv, Nq, Nk, scale, \
+                    causal, stream, device
   if (D == 128)
-    return bf16 ? launch_typed<128, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal,
-                                          stream, device)
-                : launch_typed<128, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal,
-                                           stream, device);
+    return bf16 ? launch_typed<128, true>(FA_FWD_ARGS) : launch_typed<128, false>(FA_FWD_ARGS);
   if (D == 64)
-    return bf16 ? launch_typed<64, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal,
-                                         stream, device)
-                : launch_typed<64, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal,
-                                          stream, device);
-  return set_error(FA_ERR_UNSUPPORTED, "head dimension %d is not supported (64 or 128)", D);
+    return bf16 ? launch_typed<64, true>(FA_FWD_ARGS) : launch_typed<64, false>(FA_FWD_ARGS);
+#undef FA_FWD_ARGS
+  return set_error(FA_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", D);
 }
 
 }  // namespace fa

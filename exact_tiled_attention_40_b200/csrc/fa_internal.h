@@ -26,7 +26,11 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 // Forward prefill launcher (validated arguments).  bf16 selects bf16 inputs,
 // otherwise fp16.  Returns an FA_* status.
-int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+// cu_q == nullptr: dense [B, H, N, D] tensors; otherwise a ragged batch packed as
+// [total, H, D] with per-sequence row offsets cu_q / cu_k ([B + 1], device) and
+// Nq / Nk bounding the sequence lengths.
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+               const int* cu_q, const int* cu_k, int total_q, int total_k, int B, int Hq,
                int Hkv, int Nq, int Nk, int D, float scale, int causal, bool bf16,
                cudaStream_t stream, int device);
 

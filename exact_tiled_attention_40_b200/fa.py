@@ -29,6 +29,10 @@ _F = ctypes.c_float
 _SIGS = {
     "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_fwd_fp16": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_fwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I,
+                           _P]),
+    "fa_fwd_varlen_fp16": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
+                                _I, _P]),
     "fa_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _I, _I, _P]),
     "fa_decode_paged_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _I, _I,
                                      _P]),
@@ -103,6 +107,41 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | 
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device) if return_lse else None
     fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D, scale, causal)
+    return o, lse
+
+
+def fa_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, B, Hq, Hkv, max_q, max_k, total_q, total_k, D,
+                  scale, causal, stream=None):
+    """Raw call of the ragged-batch entry point (bf16 or fp16 chosen from q's dtype)."""
+    fn = lib().fa_fwd_varlen if q.dtype == torch.bfloat16 else lib().fa_fwd_varlen_fp16
+    s = _stream(q.device) if stream is None else ctypes.c_void_p(stream)
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_q), _ptr(cu_k), B, Hq, Hkv,
+              max_q, max_k, total_q, total_k, D, float(scale), int(bool(causal)), s),
+           "fa_fwd_varlen")
+
+
+def attention_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: torch.Tensor,
+                     cu_seqlens_k: torch.Tensor, max_seqlen_q: int, max_seqlen_k: int,
+                     scale: float | None = None, causal: bool = False, return_lse: bool = True):
+    """O [total_q,Hq,D] (and LSE [Hq,total_q]) for a ragged batch packed as
+    q [total_q,Hq,D], k, v [total_k,Hkv,D] with int32 offsets cu_seqlens_* [B+1]."""
+    for t in (q, k, v, cu_seqlens_q, cu_seqlens_k):
+        if not t.is_cuda:
+            raise FAError(1, "attention_varlen", "tensors must live on a CUDA device")
+    if q.dtype not in (torch.bfloat16, torch.float16) or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise FAError(1, "attention_varlen", "q, k, v must share dtype bf16 or fp16")
+    if cu_seqlens_q.dtype != torch.int32 or cu_seqlens_k.dtype != torch.int32:
+        raise FAError(1, "attention_varlen", "cu_seqlens must be int32")
+    q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+    total_q, Hq, D = q.shape
+    total_k, Hkv, _ = k.shape
+    B = cu_seqlens_q.numel() - 1
+    if scale is None:
+        scale = D ** -0.5
+    o = torch.empty_like(q)
+    lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device) if return_lse else None
+    fa_fwd_varlen(q, k, v, o, lse, cu_seqlens_q.contiguous(), cu_seqlens_k.contiguous(), B, Hq,
+                  Hkv, int(max_seqlen_q), int(max_seqlen_k), total_q, total_k, D, scale, causal)
     return o, lse
 
 

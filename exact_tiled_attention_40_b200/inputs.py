@@ -17,6 +17,11 @@ sequence takes ceil(len / page_size) pages from the permutation in sequence
 order (so no page is shared); then q ``randn(B, Hq, D)``; then the K pool and
 the V pool, each drawn in chunks of 1024 pages as ``randn(c, page_size, Hkv, D)``.
 Unused block-table entries are 0.
+
+Recipe (ragged prefill): one generator seeded with the case seed; the key
+lengths ``randint(lo, hi + 1, (B,))`` unless the case lists them; query lengths
+equal to the key lengths (or listed); then packed Q [total_q, Hq, D], K and V
+[total_k, Hkv, D], each ``randn`` in fp32 rounded to the storage dtype.
 """
 from __future__ import annotations
 
@@ -25,8 +30,9 @@ from dataclasses import dataclass, field
 
 import torch
 
-__all__ = ["PrefillCase", "DecodeCase", "PREFILL_CASES", "DECODE_CASES",
-           "make_prefill", "make_decode", "sample_rows"]
+__all__ = ["PrefillCase", "DecodeCase", "VarlenCase", "PREFILL_CASES", "DECODE_CASES",
+           "VARLEN_CASES", "make_prefill", "make_decode", "make_varlen", "varlen_flops",
+           "sample_rows"]
 
 _DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16}
 
@@ -184,3 +190,71 @@ def make_decode(case: DecodeCase, with_pool: bool = True):
             pools.append(pool)
         kc, vc = pools
     return q, kc, vc, block_table, seq_lens.to(torch.int32)
+
+
+@dataclass(frozen=True)
+class VarlenCase:
+    """A ragged batch packed without padding: sequence b has nq[b] queries and
+    nk[b] keys (drawn from [lo, hi] when not listed)."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    D: int
+    dtype: str
+    causal: bool
+    seed: int
+    lo: int = 1
+    hi: int = 1
+    nq: tuple = ()
+    nk: tuple = ()
+
+    @property
+    def softmax_scale(self) -> float:
+        return 1.0 / math.sqrt(self.D)
+
+
+def varlen_lengths(case: VarlenCase, gen: torch.Generator):
+    if case.nk:
+        nk = torch.tensor(case.nk, dtype=torch.int64)
+    else:
+        nk = torch.randint(case.lo, case.hi + 1, (case.B,), generator=gen)
+    nq = torch.tensor(case.nq, dtype=torch.int64) if case.nq else nk.clone()
+    return nq, nk
+
+
+def make_varlen(case: VarlenCase):
+    """q [total_q, Hq, D], k, v [total_k, Hkv, D], cu_q, cu_k (int32 [B + 1]) on the CPU."""
+    gen = torch.Generator("cpu").manual_seed(case.seed)
+    nq, nk = varlen_lengths(case, gen)
+    dt = torch.bfloat16 if case.dtype == "bf16" else torch.float16
+    cu_q = torch.zeros(case.B + 1, dtype=torch.int32)
+    cu_k = torch.zeros(case.B + 1, dtype=torch.int32)
+    cu_q[1:] = torch.cumsum(nq, 0).to(torch.int32)
+    cu_k[1:] = torch.cumsum(nk, 0).to(torch.int32)
+    tq, tk = int(cu_q[-1]), int(cu_k[-1])
+    q = torch.randn(tq, case.Hq, case.D, generator=gen).to(dt)
+    k = torch.randn(tk, case.Hkv, case.D, generator=gen).to(dt)
+    v = torch.randn(tk, case.Hkv, case.D, generator=gen).to(dt)
+    return q, k, v, cu_q, cu_k
+
+
+def varlen_flops(cu_q, cu_k, Hq: int, D: int, causal: bool) -> float:
+    """4 * Hq * D * (visible query-key pairs) summed over the sequences."""
+    total = 0
+    for b in range(len(cu_q) - 1):
+        nq = int(cu_q[b + 1] - cu_q[b])
+        nk = int(cu_k[b + 1] - cu_k[b])
+        if causal:
+            # query i sees keys 0 .. i + nk - nq
+            total += sum(min(nk, i + nk - nq + 1) for i in range(nq)) if nq else 0
+        else:
+            total += nq * nk
+    return 4.0 * Hq * D * total
+
+
+VARLEN_CASES = {
+    # a serving-like mix: 16 sequences, lengths U[256, 8192], Llama-3-8B heads, causal
+    "varlen_b16_hq32_hkv8_d128_causal": VarlenCase("varlen_b16_hq32_hkv8_d128_causal", 16, 32, 8,
+                                                    128, "bf16", True, seed=5, lo=256, hi=8192),
+}

@@ -17,13 +17,14 @@ import statistics
 import torch
 
 from . import fa
-from .inputs import DECODE_CASES, PREFILL_CASES, make_decode, make_prefill
+from .inputs import (DECODE_CASES, PREFILL_CASES, VARLEN_CASES, make_decode, make_prefill,
+                     make_varlen, varlen_flops)
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--case", required=True,
-                    choices=sorted(PREFILL_CASES) + sorted(DECODE_CASES))
+                    choices=sorted(PREFILL_CASES) + sorted(DECODE_CASES) + sorted(VARLEN_CASES))
     ap.add_argument("--iters", type=int, default=5)
     args = ap.parse_args()
     dev = torch.device("cuda", 0)
@@ -40,6 +41,21 @@ def main():
             fa.fa_fwd(q, k, v, o, lse, c.B, c.Hq, c.Hkv, c.Nq, c.Nk, c.D, c.softmax_scale,
                       c.causal, stream=stream.cuda_stream)
         work, unit = c.flops / 1e12, "TFLOP/s"
+    elif args.case in VARLEN_CASES:
+        c = VARLEN_CASES[args.case]
+        q, k, v, cu_q, cu_k = make_varlen(c)
+        flops = varlen_flops(cu_q, cu_k, c.Hq, c.D, c.causal)
+        max_q = int((cu_q[1:] - cu_q[:-1]).max())
+        max_k = int((cu_k[1:] - cu_k[:-1]).max())
+        q, k, v, cu_q, cu_k = (t.to(dev) for t in (q, k, v, cu_q, cu_k))
+        o = torch.empty_like(q)
+        lse = torch.empty((c.Hq, q.shape[0]), dtype=torch.float32, device=dev)
+
+        def launch():
+            fa.fa_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, c.B, c.Hq, c.Hkv, max_q, max_k,
+                             q.shape[0], k.shape[0], c.D, c.softmax_scale, c.causal,
+                             stream=stream.cuda_stream)
+        work, unit = flops / 1e12, "TFLOP/s"
     else:
         c = DECODE_CASES[args.case]
         q, kc, vc, table, lens = make_decode(c)

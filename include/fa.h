@@ -77,6 +77,40 @@ int fa_fwd_fp16(const void* q, const void* k, const void* v, void* o, float* lse
                 int Hkv, int Nq, int Nk, int D, float scale, int causal, fa_stream_t stream);
 
 /*
+ * Prefill over a ragged batch packed without padding (bf16).
+ *
+ * Sequence b owns query rows [cu_seqlens_q[b], cu_seqlens_q[b+1]) and key rows
+ * [cu_seqlens_k[b], cu_seqlens_k[b+1]); its queries see only its own keys.
+ * This is the padded batch of devhandbook.co.kr "Flash Attention 2 ... PyTorch
+ * native", example 3 (causal rule with a padding mask) without the padding, for
+ * the length-mixed batches of cabseo.com "Advanced techniques for enhancing LLM
+ * throughput", section "Continuous batching".
+ *   q   [total_q, Hq,  D] bf16        k, v [total_k, Hkv, D] bf16
+ *   o   [total_q, Hq,  D] bf16 (written rows of valid sequences only)
+ *   lse [Hq, total_q]     fp32 (written; may be NULL), as for fa_fwd
+ *   cu_seqlens_q, cu_seqlens_k  [B + 1] int32 on the device, non-decreasing,
+ *       starting at 0 and ending at most at total_q / total_k.
+ *   max_seqlen_q, max_seqlen_k  bounds on every sequence's lengths (the grid is
+ *       sized from max_seqlen_q).
+ * causal: bottom-right aligned within each sequence; needs Nq_b <= Nk_b.
+ * GQA, D, scale and the empty cases as for fa_fwd; a sequence with no keys gets
+ * O = 0 and LSE = -inf.  The host cannot read the offsets: a sequence whose
+ * offsets break these rules (or whose length exceeds the bound) is skipped, its
+ * rows are not written, and FA_ERR_DEVICE_INDEX is raised in fa_device_status().
+ * No workspace is allocated.
+ */
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B, int Hq,
+                  int Hkv, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int D,
+                  float scale, int causal, fa_stream_t stream);
+
+/* Same as fa_fwd_varlen with fp16 q, k, v and o (fp32 LSE). */
+int fa_fwd_varlen_fp16(const void* q, const void* k, const void* v, void* o, float* lse,
+                       const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B, int Hq,
+                       int Hkv, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+                       int D, float scale, int causal, fa_stream_t stream);
+
+/*
  * Decode over a paged KV cache: one new query token per sequence attends over
  * all of that sequence's cached keys and values (no mask beyond its length).
  *   q           [B, Hq, D] bf16
@@ -93,7 +127,7 @@ int fa_fwd_fp16(const void* q, const void* k, const void* v, void* o, float* lse
  * of range are skipped and flagged in the device error word.
  * A sequence of length 0 gets O = 0 and LSE = -inf.
  * Work is split over key chunks; partial results are merged by their LSE.
- * For Hkv <= 8 and Hq/Hkv <= 4 one persistent CTA per SM takes an equal share of all
+ * For Hkv <= 8 one persistent CTA per SM takes an equal share of all
  * sequences' cache (so ragged lengths stay balanced); otherwise the grid is
  * (chunk, sequence).  The partials live in a stream-ordered workspace taken
  * from a library-owned memory pool on `stream` and returned to it on `stream`

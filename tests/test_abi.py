@@ -80,3 +80,32 @@ def test_valid_call_without_a_device_fails_loudly(lib):
     assert dec(lib) == E["FA_ERR_NO_DEVICE"]
     with pytest.raises(fa.FAError):
         fa._check(fwd(lib), "fa_fwd")
+
+
+def varlen(lib, B=2, Hq=4, Hkv=2, max_q=9, max_k=9, tq=12, tk=14, D=128, scale=0.1, causal=0,
+           q=FAKE, k=FAKE, v=FAKE, o=FAKE, cuq=FAKE, cuk=FAKE):
+    return lib.fa_fwd_varlen(q, k, v, o, None, cuq, cuk, B, Hq, Hkv, max_q, max_k, tq, tk, D,
+                             scale, causal, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=-1), "FA_ERR_INVALID_ARG"),
+    (dict(tq=-3), "FA_ERR_INVALID_ARG"),
+    (dict(D=80), "FA_ERR_UNSUPPORTED"),
+    (dict(Hq=5), "FA_ERR_INVALID_ARG"),
+    (dict(cuq=None), "FA_ERR_INVALID_ARG"),
+    (dict(cuk=None), "FA_ERR_INVALID_ARG"),
+    (dict(k=None), "FA_ERR_INVALID_ARG"),
+    (dict(q=FAKE + 2), "FA_ERR_INVALID_ARG"),
+    (dict(scale=-1.0), "FA_ERR_INVALID_ARG"),
+])
+def test_varlen_rejects_bad_arguments_on_the_host(lib, kw, code):
+    assert varlen(lib, **kw) == E[code]
+    assert lib.fa_last_error_string()
+
+
+def test_varlen_empty_batch_is_a_noop(lib):
+    assert varlen(lib, B=0) == 0
+    assert varlen(lib, tq=0) == 0
+    assert varlen(lib, max_q=0) == 0
+    assert varlen(lib, tk=0, k=None, v=None, q=FAKE) in (0, E["FA_ERR_NO_DEVICE"])
