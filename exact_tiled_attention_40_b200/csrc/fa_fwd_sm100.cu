@@ -101,33 +101,41 @@ __device__ __forceinline__ int kv_tiles_for(int first_row, int Nq, int Nk, int c
   return min(nk_tiles, max_key / kBN + 1);
 }
 
-// Work item i: (batch, head, pair of 128-row query tiles); with a causal mask the
-// pairs are ordered heaviest first.
+// A work item: (sequence b, query head h, pair of 128-row query tiles).
 struct FwdItem {
   int bh, b, h, hkv, q_row0, n0, n1;
   int q_start, k_start, nq, nk;   // the sequence's rows (dense: 0, 0, Nq, Nk)
-  bool bad;                       // ragged offsets out of range: the item is skipped
 };
-__device__ __forceinline__ FwdItem item_of(int i, const FwdParams& p) {
+
+// Rows of sequence b of a ragged batch, or false when its offsets break the rules
+// (negative length, past the packed tensor, longer than the bound, causal with
+// more queries than keys).
+__device__ __forceinline__ bool ragged_rows(const FwdParams& p, int b, int& q0, int& nq, int& k0,
+                                            int& nk) {
+  q0 = __ldg(p.cu_q + b);
+  const int q1 = __ldg(p.cu_q + b + 1);
+  k0 = __ldg(p.cu_k + b);
+  const int k1 = __ldg(p.cu_k + b + 1);
+  nq = q1 - q0;
+  nk = k1 - k0;
+  return q0 >= 0 && nq >= 0 && q1 <= p.total_q && nq <= p.Nq && k0 >= 0 && nk >= 0 &&
+         k1 <= p.total_k && !(p.causal && nq > nk);
+}
+__device__ __forceinline__ int ragged_pairs(const FwdParams& p, int b) {
+  int q0, nq, k0, nk;
+  return ragged_rows(p, b, q0, nq, k0, nk) ? (nq + 2 * kBM - 1) / (2 * kBM) : 0;
+}
+
+template <bool RAGGED>
+__device__ __forceinline__ FwdItem make_item(const FwdParams& p, int b, int h, int mpair) {
   FwdItem it;
-  const int BH = p.B * p.Hq;
-  const int mrev = i / BH;
-  it.bh = i - mrev * BH;
-  const int mpair = p.causal ? (p.num_mpairs - 1 - mrev) : mrev;
-  it.b = it.bh / p.Hq;
-  it.h = it.bh - it.b * p.Hq;
-  it.hkv = it.h / (p.Hq / p.Hkv);
+  it.b = b;
+  it.h = h;
+  it.bh = b * p.Hq + h;
+  it.hkv = h / (p.Hq / p.Hkv);
   it.q_row0 = mpair * 2 * kBM;
-  it.bad = false;
-  if (p.cu_q) {
-    const int q0 = p.cu_q[it.b], q1 = p.cu_q[it.b + 1];
-    const int k0 = p.cu_k[it.b], k1 = p.cu_k[it.b + 1];
-    it.bad = q0 < 0 || q1 < q0 || q1 > p.total_q || q1 - q0 > p.Nq || k0 < 0 || k1 < k0 ||
-             k1 > p.total_k || (p.causal && q1 - q0 > k1 - k0);
-    it.q_start = q0;
-    it.k_start = k0;
-    it.nq = it.bad ? 0 : q1 - q0;
-    it.nk = it.bad ? 0 : k1 - k0;
+  if constexpr (RAGGED) {
+    if (!ragged_rows(p, b, it.q_start, it.nq, it.k_start, it.nk)) it.nq = it.nk = 0;
   } else {
     it.q_start = 0;
     it.k_start = 0;
@@ -138,15 +146,84 @@ __device__ __forceinline__ FwdItem item_of(int i, const FwdParams& p) {
   it.n1 = kv_tiles_for(it.q_row0 + kBM, it.nq, it.nk, p.causal);
   return it;
 }
-// The r-th item of CTA c: rounds of gridDim items, alternately left to right and
-// right to left (with the heaviest-first order this balances the CTAs' totals
-// about as well as handing items out dynamically); -1 when none is left.
-__device__ __forceinline__ int item_index(int c, int r, int C, int total) {
-  const int i = r * C + ((r & 1) ? C - 1 - c : c);
-  return i < total ? i : -1;
-}
 
-template <int D, bool BF16>
+// The items of one CTA, in order.  The list is ordered by tile pair (heaviest
+// first when causal), then sequence, then head; CTA c takes the r-th entry of
+// rounds of gridDim entries, alternately left to right and right to left (with
+// the heaviest-first order this balances the CTAs' totals about as well as
+// handing items out dynamically).  Dense batches index the list in closed form.
+// Ragged batches list only pairs that start inside their sequence (pair m of
+// sequence b for m < ceil(Nq_b / 256)), so the rounds contain no empty items;
+// every role of the CTA walks a cursor along that list, whose indices only grow.
+// (Separate instantiations keep the dense kernel free of the cursor.)
+template <bool RAGGED>
+struct ItemWalker {
+  int cta, C, r, total;
+  int idx, m, b, h;   // ragged cursor: list entry idx is (pair m, sequence b, head h)
+
+  __device__ void init(const FwdParams& p, int cta_, int C_) {
+    cta = cta_;
+    C = C_;
+    r = 0;
+    if constexpr (!RAGGED) {
+      total = p.num_items;
+      return;
+    }
+    int sum = 0, pmax = 0;
+    for (int bb = 0; bb < p.B; ++bb) {
+      const int pb = ragged_pairs(p, bb);
+      sum += pb;
+      pmax = max(pmax, pb);
+    }
+    total = sum * p.Hq;
+    idx = 0;
+    h = 0;
+    m = pmax - 1;
+    b = 0;
+    if (total > 0)
+      while (ragged_pairs(p, b) <= m) ++b;
+  }
+  // Moves the ragged cursor to list entry `target` (>= idx, < total).
+  __device__ void advance(const FwdParams& p, int target) {
+    int k = target - idx;
+    while (k > 0) {
+      const int left = p.Hq - h;
+      if (k < left) {
+        h += k;
+        break;
+      }
+      k -= left;
+      h = 0;
+      do {
+        ++b;
+      } while (b < p.B && ragged_pairs(p, b) <= m);
+      if (b == p.B) {                            // next (lighter) pair of every sequence
+        --m;
+        b = 0;
+        while (b < p.B && ragged_pairs(p, b) <= m) ++b;
+      }
+    }
+    idx = target;
+  }
+  __device__ bool next(const FwdParams& p, FwdItem& it) {
+    const int i = r * C + ((r & 1) ? C - 1 - cta : cta);
+    ++r;
+    if (i >= total) return false;
+    if constexpr (RAGGED) {
+      advance(p, i);
+      it = make_item<true>(p, b, h, m);
+    } else {
+      const int BH = p.B * p.Hq;
+      const int mrev = i / BH;
+      const int bh = i - mrev * BH;
+      const int b_ = bh / p.Hq;
+      it = make_item<false>(p, b_, bh - b_ * p.Hq, p.causal ? (p.num_mpairs - 1 - mrev) : mrev);
+    }
+    return true;
+  }
+};
+
+template <int D, bool BF16, bool RAGGED>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -177,6 +254,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
+  if (RAGGED && cta == 0 && tid == 0) {
+    for (int b = 0; b < p.B; ++b) {
+      int q0, nq, k0, nk;
+      if (!ragged_rows(p, b, q0, nq, k0, nk)) {
+        atomicOr(p.err, kErrBadIndex);           // that sequence is skipped
+        break;
+      }
+    }
+  }
   if (tid == 0) {
     for (int t = 0; t < 2; ++t) {
       mbar_init(q_full(t), 1);
@@ -214,10 +300,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmV);
         int pos = 0, items = 0;
         bool ok = true;
-        for (int r = 0; ok; ++r) {
-          const int i = item_index(cta, r, C, p.num_items);
-          if (i < 0) break;
-          const FwdItem it = item_of(i, p);
+        ItemWalker<RAGGED> walk;
+        walk.init(p, cta, C);
+        FwdItem it;
+        while (ok && walk.next(p, it)) {
           const int n_max = max(it.n0, it.n1);
           if (n_max == 0) continue;
           if (items > 0 && !mbar_wait(q_empty, (items - 1) & 1, abort_flag, p.err, p.timeout_ns))
@@ -226,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(q_full(t), L::kTileBytes);
             const uint32_t dst = sbase + L::kQOff + t * L::kTileBytes;
             for (int ch = 0; ch < L::kChunks; ++ch) {
-              if (p.cu_q)   // [total_q, Hq, D]: box {64, 1 head, 128 rows}
+              if (RAGGED)   // [total_q, Hq, D]: box {64, 1 head, 128 rows}
                 tma_load_3d(dst + ch * L::kChunkBytes, &tmQ, q_full(t), ch * 64, it.h,
                             it.q_start + it.q_row0 + t * kBM);
               else          // [B * Hq, Nq, D]: box {64, 128 rows, 1}
@@ -248,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t dst = sbase + L::kKVOff + slot * L::kTileBytes;
               const void* tm = w ? static_cast<const void*>(&tmV) : static_cast<const void*>(&tmK);
               for (int ch = 0; ch < L::kChunks; ++ch) {
-                if (p.cu_q)
+                if (RAGGED)
                   tma_load_3d(dst + ch * L::kChunkBytes, tm, kv_full(slot), ch * 64, it.hkv,
                               it.k_start + j * kBN);
                 else
@@ -323,10 +409,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         int pos = 0, items = 0;
         int tiles[2] = {0, 0};   // S tiles of each query-tile slot in earlier items (phases)
-        for (int r = 0; ok; ++r) {
-          const int i = item_index(cta, r, C, p.num_items);
-          if (i < 0) break;
-          const FwdItem it = item_of(i, p);
+        ItemWalker<RAGGED> walk;
+        walk.init(p, cta, C);
+        FwdItem it;
+        while (ok && walk.next(p, it)) {
           const int n_max = max(it.n0, it.n1);
           if (n_max == 0) continue;
           ok = wait(q_full(0), items & 1);
@@ -395,19 +481,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tmem + lane_base + 256 + t * D;
     int tiles = 0, outs = 0;     // S tiles and O tiles of this slot in earlier items (phases)
     bool ok = true;
-    for (int ri = 0; ok; ++ri) {
-    const int item = item_index(cta, ri, C, p.num_items);
-    if (item < 0) break;
-    const FwdItem it = item_of(item, p);
+    ItemWalker<RAGGED> walk;
+    walk.init(p, cta, C);
+    FwdItem it;
+    while (ok && walk.next(p, it)) {
     const int q_row0 = it.q_row0;
     const int row = q_row0 + t * kBM + r;          // within the sequence
     const int n = t ? it.n1 : it.n0;
-    if (it.bad && t == 0 && r == 0 && q_row0 == 0) atomicOr(p.err, kErrBadIndex);
     // o element offset / D and lse offset of this row
-    const size_t o_index = p.cu_q
+    const size_t o_index = RAGGED
         ? static_cast<size_t>(it.q_start + row) * p.Hq + it.h
         : static_cast<size_t>(it.bh) * p.Nq + row;
-    const size_t row_index = p.cu_q
+    const size_t row_index = RAGGED
         ? static_cast<size_t>(it.h) * p.total_q + it.q_start + row
         : o_index;
     using Out = uint16_t;
@@ -632,9 +717,12 @@ int launch_typed(const void* q, const void* k, const void* v, void* o, float* ls
     std::lock_guard<std::mutex> g(mu);
     if (device < 0 || device >= 64) return set_error(FA_ERR_CUDA, "device ordinal out of range");
     if (!attr_done[device]) {
-      cudaError_t e = cudaFuncSetAttribute(fa_fwd_kernel<D, BF16>,
+      cudaError_t e = cudaFuncSetAttribute(fa_fwd_kernel<D, BF16, false>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            L::kSmemBytes);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(fa_fwd_kernel<D, BF16, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
       if (e != cudaSuccess)
         return set_error(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
       attr_done[device] = true;
@@ -683,8 +771,12 @@ int launch_typed(const void* q, const void* k, const void* v, void* o, float* ls
   if (nsm <= 0) return set_error(FA_ERR_CUDA, "cannot read the SM count of device %d", device);
   const int grid = static_cast<int>(std::min<long long>(items, nsm));
   if (grid == 0) return FA_OK;
-  fa_fwd_kernel<D, BF16><<<static_cast<unsigned>(grid), kThreads, L::kSmemBytes, stream>>>(
-      tq, tk, tv, prm);
+  if (cu_q)
+    fa_fwd_kernel<D, BF16, true><<<static_cast<unsigned>(grid), kThreads, L::kSmemBytes,
+                                   stream>>>(tq, tk, tv, prm);
+  else
+    fa_fwd_kernel<D, BF16, false><<<static_cast<unsigned>(grid), kThreads, L::kSmemBytes,
+                                    stream>>>(tq, tk, tv, prm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(FA_ERR_CUDA, "fa_fwd launch: %s", cudaGetErrorString(e));
   return FA_OK;
