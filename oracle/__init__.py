@@ -12,6 +12,7 @@ from .attention_fp64 import (  # noqa: F401
     gather_paged_kv,
     kv_head_of,
     merge_partials,
+    paged_prefill,
     softmax_rows,
     varlen_attention,
 )

@@ -323,3 +323,39 @@ def varlen_attention(q, k, v, cu_seqlens_q, cu_seqlens_k, scale: float, causal: 
         O[q0:q1] = np.transpose(o[0], (1, 0, 2))
         LSE[:, q0:q1] = lse[0]
     return O, LSE
+
+
+def paged_prefill(q, kcache, vcache, block_table, cu_seqlens_q, seq_lens_k, scale: float,
+                  causal: bool, page_size: int):
+    """Prefill of new query tokens against keys/values held in a paged cache.
+
+    [cabseo] "Paged attention" (the cache is reached page by page through a
+    block table) combined with the ragged batches of ``varlen_attention``:
+    sequence b's queries are rows [cu_seqlens_q[b], cu_seqlens_q[b+1]) of q and
+    its keys are the first seq_lens_k[b] tokens of its pages.  Reading: with
+    ``causal`` the queries are the last Nq_b tokens of the sequence (bottom-right
+    alignment), as when a prompt is prefilled in chunks.
+
+    q [total_q, Hq, D]; kcache, vcache [num_pages, page_size, Hkv, D];
+    block_table [B, max_pages] int; cu_seqlens_q [B + 1]; seq_lens_k [B].
+    Returns O [total_q, Hq, D] and LSE [Hq, total_q].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    cq = np.asarray(cu_seqlens_q, dtype=np.int64)
+    lens = np.asarray(seq_lens_k, dtype=np.int64)
+    B = len(cq) - 1
+    total_q, Hq, D = q.shape
+    O = np.zeros((total_q, Hq, D))
+    LSE = np.full((Hq, total_q), -np.inf)
+    for b in range(B):
+        q0, q1 = cq[b], cq[b + 1]
+        if q1 == q0:
+            continue
+        n = int(lens[b])
+        kb = gather_paged_kv(kcache, block_table, n, b, page_size)[None]   # [1, Hkv, n, D]
+        vb = gather_paged_kv(vcache, block_table, n, b, page_size)[None]
+        qb = np.transpose(q[q0:q1], (1, 0, 2))[None]
+        o, lse = attention(qb, kb, vb, scale, causal)
+        O[q0:q1] = np.transpose(o[0], (1, 0, 2))
+        LSE[:, q0:q1] = lse[0]
+    return O, LSE

@@ -354,3 +354,32 @@ def test_pins_catch_a_varlen_offset_mixup():
     cu_bad[1:-1] = cu_q[1:-1]                 # keys split at the query boundaries
     O_bad, _ = oracle.varlen_attention(q, k, v, cu_q, cu_bad, 0.5, False)
     assert np.max(np.abs(O_bad - O_ref)) > 1e-3
+
+
+def test_paged_prefill_equals_contiguous_ragged_attention():
+    """Keys and values scattered into random pages of a pool (by the test, with
+    plain indexing) and read back through the block table give the same result
+    as the contiguous ragged batch."""
+    rng = np.random.default_rng(100)
+    page, Hq, Hkv, D = 4, 4, 2, 8
+    Nk = np.array([9, 4, 13])
+    Nq = np.array([3, 4, 5])                      # the last Nq_b tokens are the queries
+    q, k, v, cu_q, cu_k = _packed_case(Nq, Nk, Hq, Hkv, D, 101)
+    npages = [int(math.ceil(n / page)) for n in Nk]
+    pool = 20
+    perm = rng.permutation(pool)
+    table = np.zeros((3, max(npages)), dtype=np.int64)
+    kc = rng.standard_normal((pool, page, Hkv, D))      # other pages hold unrelated values
+    vc = rng.standard_normal((pool, page, Hkv, D))
+    used = 0
+    for b in range(3):
+        table[b, :npages[b]] = perm[used:used + npages[b]]
+        used += npages[b]
+        for t in range(Nk[b]):
+            kc[table[b, t // page], t % page] = k[cu_k[b] + t]
+            vc[table[b, t // page], t % page] = v[cu_k[b] + t]
+    for causal in (False, True):
+        O, L = oracle.paged_prefill(q, kc, vc, table, cu_q, Nk, 0.5, causal, page)
+        O_ref, L_ref = _padded_library(q, k, v, cu_q, cu_k, 0.5, causal)
+        np.testing.assert_allclose(O, O_ref, atol=TIGHT)
+        np.testing.assert_allclose(L, L_ref, atol=TIGHT)
