@@ -137,8 +137,8 @@ int fwd_common(const void* q, const void* k, const void* v, void* o, float* lse,
   if (B == 0 || Hq == 0 || Nq == 0) return FA_OK;
   int dev;
   if ((rc = current_sm100(&dev)) != FA_OK) return rc;
-  return launch_fwd(q, k, v, o, lse, nullptr, nullptr, 0, 0, B, Hq, Hkv, Nq, Nk, D, scale, causal,
-                    bf16, stream, dev);
+  return launch_fwd(q, k, v, o, lse, FwdLayoutArgs{}, B, Hq, Hkv, Nq, Nk, D, scale, causal, bf16,
+                    stream, dev);
 }
 
 int varlen_common(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -165,8 +165,55 @@ int varlen_common(const void* q, const void* k, const void* v, void* o, float* l
     return set_error(FA_ERR_INVALID_ARG, "total_q * Hq too large");
   int dev, rc;
   if ((rc = current_sm100(&dev)) != FA_OK) return rc;
-  return launch_fwd(q, k, v, o, lse, cu_q, cu_k, total_q, total_k, B, Hq, Hkv, max_seqlen_q,
-                    max_seqlen_k, D, scale, causal, bf16, stream, dev);
+  FwdLayoutArgs la;
+  la.cu_q = cu_q;
+  la.cu_k = cu_k;
+  la.total_q = total_q;
+  la.total_k = total_k;
+  return launch_fwd(q, k, v, o, lse, la, B, Hq, Hkv, max_seqlen_q, max_seqlen_k, D, scale, causal,
+                    bf16, stream, dev);
+}
+
+int paged_common(const void* q, const void* kcache, const void* vcache,
+                 const int32_t* block_table, void* o, float* lse, const int32_t* cu_q,
+                 const int32_t* seq_lens_k, int B, int Hq, int Hkv, int max_seqlen_q,
+                 int max_pages_per_seq, int num_pages, int total_q, int D, int page_size,
+                 float scale, int causal, cudaStream_t stream, bool bf16) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || max_seqlen_q < 0 || max_pages_per_seq < 0 ||
+      num_pages < 0 || total_q < 0)
+    return set_error(FA_ERR_INVALID_ARG, "negative size");
+  if (!(std::isfinite(scale) && scale > 0.f))
+    return set_error(FA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (D != 64 && D != 128)
+    return set_error(FA_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", D);
+  if (page_size != 16)
+    return set_error(FA_ERR_UNSUPPORTED, "paged prefill supports page_size == 16 only (got %d)",
+                     page_size);
+  if (B == 0 || Hq == 0 || total_q == 0 || max_seqlen_q == 0) return FA_OK;
+  if (Hkv <= 0 || Hq % Hkv != 0)
+    return set_error(FA_ERR_INVALID_ARG, "Hq (%d) must be a positive multiple of Hkv (%d)", Hq,
+                     Hkv);
+  if (max_pages_per_seq <= 0 || num_pages <= 0)
+    return set_error(FA_ERR_INVALID_ARG, "max_pages_per_seq and num_pages must be positive");
+  if (!q || !kcache || !vcache || !block_table || !o || !cu_q || !seq_lens_k)
+    return set_error(FA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o))
+    return set_error(FA_ERR_INVALID_ARG, "q, caches and o must be 16-byte aligned");
+  if (static_cast<long long>(max_pages_per_seq) * 16 > 0x7fffffffLL ||
+      static_cast<long long>(num_pages) * 16 > 0x7fffffffLL ||
+      static_cast<long long>(total_q) * Hq > 0x7fffffffLL)
+    return set_error(FA_ERR_INVALID_ARG, "sizes too large");
+  int dev, rc;
+  if ((rc = current_sm100(&dev)) != FA_OK) return rc;
+  FwdLayoutArgs la;
+  la.cu_q = cu_q;
+  la.total_q = total_q;
+  la.block_table = block_table;
+  la.seq_lens_k = seq_lens_k;
+  la.max_pages = max_pages_per_seq;
+  la.num_pages = num_pages;
+  return launch_fwd(q, kcache, vcache, o, lse, la, B, Hq, Hkv, max_seqlen_q,
+                    max_pages_per_seq * 16, D, scale, causal, bf16, stream, dev);
 }
 
 }  // namespace
@@ -202,6 +249,16 @@ int fa_fwd_varlen_fp16(const void* q, const void* k, const void* v, void* o, flo
   return fa::varlen_common(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, Hq, Hkv, max_seqlen_q,
                            max_seqlen_k, total_q, total_k, D, scale, causal,
                            reinterpret_cast<cudaStream_t>(stream), false);
+}
+
+int fa_fwd_paged(const void* q, const void* kcache, const void* vcache,
+                 const int32_t* block_table, void* o, float* lse, const int32_t* cu_seqlens_q,
+                 const int32_t* seq_lens_k, int B, int Hq, int Hkv, int max_seqlen_q,
+                 int max_pages_per_seq, int num_pages, int total_q, int D, int page_size,
+                 float scale, int causal, fa_stream_t stream) {
+  return fa::paged_common(q, kcache, vcache, block_table, o, lse, cu_seqlens_q, seq_lens_k, B, Hq,
+                          Hkv, max_seqlen_q, max_pages_per_seq, num_pages, total_q, D, page_size,
+                          scale, causal, reinterpret_cast<cudaStream_t>(stream), true);
 }
 
 int fa_decode_paged(const void* q, const void* kcache, const void* vcache,

@@ -81,6 +81,11 @@ struct FwdParams {
   const int* cu_q;
   const int* cu_k;
   int total_q, total_k;
+  // Paged keys/values (cu_k unused): sequence b's keys are the first seq_lens_k[b]
+  // tokens of its pages block_table[b][0 ..] in the pool k/v [num_pages, 16, Hkv, D].
+  const int* block_table;
+  const int* seq_lens_k;
+  int max_pages, num_pages;
   int B, Hq, Hkv, Nq, Nk;
   int num_mpairs;
   int num_items;      // num_mpairs * B * Hq work items, heaviest first
@@ -107,26 +112,41 @@ struct FwdItem {
   int q_start, k_start, nq, nk;   // the sequence's rows (dense: 0, 0, Nq, Nk)
 };
 
-// Rows of sequence b of a ragged batch, or false when its offsets break the rules
-// (negative length, past the packed tensor, longer than the bound, causal with
-// more queries than keys).
+// Batch layouts (kernel instantiations): dense [B, H, N, D]; ragged (packed
+// [total, H, D] queries and keys with row offsets); paged (packed queries, keys
+// and values in a page pool reached through a block table).
+enum : int { kDense = 0, kRagged = 1, kPaged = 2 };
+constexpr int kPageTok = 16;   // tokens per page of a paged pool
+
+// Rows of sequence b of a ragged or paged batch, or false when its offsets or
+// length break the rules (negative length, past the packed tensor or the block
+// table, longer than the bound, causal with more queries than keys).
+template <int MODE>
 __device__ __forceinline__ bool ragged_rows(const FwdParams& p, int b, int& q0, int& nq, int& k0,
                                             int& nk) {
   q0 = __ldg(p.cu_q + b);
   const int q1 = __ldg(p.cu_q + b + 1);
-  k0 = __ldg(p.cu_k + b);
-  const int k1 = __ldg(p.cu_k + b + 1);
   nq = q1 - q0;
-  nk = k1 - k0;
-  return q0 >= 0 && nq >= 0 && q1 <= p.total_q && nq <= p.Nq && k0 >= 0 && nk >= 0 &&
-         k1 <= p.total_k && !(p.causal && nq > nk);
+  bool ok = q0 >= 0 && nq >= 0 && q1 <= p.total_q && nq <= p.Nq;
+  if constexpr (MODE == kPaged) {
+    k0 = 0;
+    nk = __ldg(p.seq_lens_k + b);
+    ok = ok && nk >= 0 && nk <= p.max_pages * kPageTok;
+  } else {
+    k0 = __ldg(p.cu_k + b);
+    const int k1 = __ldg(p.cu_k + b + 1);
+    nk = k1 - k0;
+    ok = ok && k0 >= 0 && nk >= 0 && k1 <= p.total_k;
+  }
+  return ok && !(p.causal && nq > nk);
 }
+template <int MODE>
 __device__ __forceinline__ int ragged_pairs(const FwdParams& p, int b) {
   int q0, nq, k0, nk;
-  return ragged_rows(p, b, q0, nq, k0, nk) ? (nq + 2 * kBM - 1) / (2 * kBM) : 0;
+  return ragged_rows<MODE>(p, b, q0, nq, k0, nk) ? (nq + 2 * kBM - 1) / (2 * kBM) : 0;
 }
 
-template <bool RAGGED>
+template <int MODE>
 __device__ __forceinline__ FwdItem make_item(const FwdParams& p, int b, int h, int mpair) {
   FwdItem it;
   it.b = b;
@@ -134,8 +154,8 @@ __device__ __forceinline__ FwdItem make_item(const FwdParams& p, int b, int h, i
   it.bh = b * p.Hq + h;
   it.hkv = h / (p.Hq / p.Hkv);
   it.q_row0 = mpair * 2 * kBM;
-  if constexpr (RAGGED) {
-    if (!ragged_rows(p, b, it.q_start, it.nq, it.k_start, it.nk)) it.nq = it.nk = 0;
+  if constexpr (MODE != kDense) {
+    if (!ragged_rows<MODE>(p, b, it.q_start, it.nq, it.k_start, it.nk)) it.nq = it.nk = 0;
   } else {
     it.q_start = 0;
     it.k_start = 0;
@@ -156,7 +176,7 @@ __device__ __forceinline__ FwdItem make_item(const FwdParams& p, int b, int h, i
 // sequence b for m < ceil(Nq_b / 256)), so the rounds contain no empty items;
 // every role of the CTA walks a cursor along that list, whose indices only grow.
 // (Separate instantiations keep the dense kernel free of the cursor.)
-template <bool RAGGED>
+template <int MODE>
 struct ItemWalker {
   int cta, C, r, total;
   int idx, m, b, h;   // ragged cursor: list entry idx is (pair m, sequence b, head h)
@@ -165,13 +185,13 @@ struct ItemWalker {
     cta = cta_;
     C = C_;
     r = 0;
-    if constexpr (!RAGGED) {
+    if constexpr (MODE == kDense) {
       total = p.num_items;
       return;
     }
     int sum = 0, pmax = 0;
     for (int bb = 0; bb < p.B; ++bb) {
-      const int pb = ragged_pairs(p, bb);
+      const int pb = ragged_pairs<MODE>(p, bb);
       sum += pb;
       pmax = max(pmax, pb);
     }
@@ -181,7 +201,7 @@ struct ItemWalker {
     m = pmax - 1;
     b = 0;
     if (total > 0)
-      while (ragged_pairs(p, b) <= m) ++b;
+      while (ragged_pairs<MODE>(p, b) <= m) ++b;
   }
   // Moves the ragged cursor to list entry `target` (>= idx, < total).
   __device__ void advance(const FwdParams& p, int target) {
@@ -196,11 +216,11 @@ struct ItemWalker {
       h = 0;
       do {
         ++b;
-      } while (b < p.B && ragged_pairs(p, b) <= m);
+      } while (b < p.B && ragged_pairs<MODE>(p, b) <= m);
       if (b == p.B) {                            // next (lighter) pair of every sequence
         --m;
         b = 0;
-        while (b < p.B && ragged_pairs(p, b) <= m) ++b;
+        while (b < p.B && ragged_pairs<MODE>(p, b) <= m) ++b;
       }
     }
     idx = target;
@@ -209,24 +229,25 @@ struct ItemWalker {
     const int i = r * C + ((r & 1) ? C - 1 - cta : cta);
     ++r;
     if (i >= total) return false;
-    if constexpr (RAGGED) {
+    if constexpr (MODE != kDense) {
       advance(p, i);
-      it = make_item<true>(p, b, h, m);
+      it = make_item<MODE>(p, b, h, m);
     } else {
       const int BH = p.B * p.Hq;
       const int mrev = i / BH;
       const int bh = i - mrev * BH;
       const int b_ = bh / p.Hq;
-      it = make_item<false>(p, b_, bh - b_ * p.Hq, p.causal ? (p.num_mpairs - 1 - mrev) : mrev);
+      it = make_item<kDense>(p, b_, bh - b_ * p.Hq, p.causal ? (p.num_mpairs - 1 - mrev) : mrev);
     }
     return true;
   }
 };
 
-template <int D, bool BF16, bool RAGGED>
+template <int D, bool BF16, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  constexpr bool RAGGED = MODE != kDense;
   using L = FwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -257,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (RAGGED && cta == 0 && tid == 0) {
     for (int b = 0; b < p.B; ++b) {
       int q0, nq, k0, nk;
-      if (!ragged_rows(p, b, q0, nq, k0, nk)) {
+      if (!ragged_rows<MODE>(p, b, q0, nq, k0, nk)) {
         atomicOr(p.err, kErrBadIndex);           // that sequence is skipped
         break;
       }
@@ -300,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmV);
         int pos = 0, items = 0;
         bool ok = true;
-        ItemWalker<RAGGED> walk;
+        ItemWalker<MODE> walk;
         walk.init(p, cta, C);
         FwdItem it;
         while (ok && walk.next(p, it)) {
@@ -333,13 +354,31 @@ __global__ void __launch_bounds__(kThreads, 1)
               mbar_arrive_expect_tx(kv_full(slot), L::kTileBytes);
               const uint32_t dst = sbase + L::kKVOff + slot * L::kTileBytes;
               const void* tm = w ? static_cast<const void*>(&tmV) : static_cast<const void*>(&tmK);
-              for (int ch = 0; ch < L::kChunks; ++ch) {
-                if (RAGGED)
-                  tma_load_3d(dst + ch * L::kChunkBytes, tm, kv_full(slot), ch * 64, it.hkv,
-                              it.k_start + j * kBN);
-                else
-                  tma_load_3d(dst + ch * L::kChunkBytes, tm, kv_full(slot), ch * 64, j * kBN,
-                              kv_z);
+              if constexpr (MODE == kPaged) {
+                // eight 16-token boxes, one per page; keys past the sequence read its
+                // first page (masked later, but finite); an id outside the pool is
+                // flagged and replaced by page 0
+                const int* tab = p.block_table + static_cast<size_t>(it.b) * p.max_pages;
+                for (int pg = 0; pg < kBN / kPageTok; ++pg) {
+                  const int tok = j * kBN + pg * kPageTok;
+                  int page = __ldg(tab + (tok < it.nk ? tok / kPageTok : 0));
+                  if (page < 0 || page >= p.num_pages) {
+                    atomicOr(p.err, kErrBadIndex);
+                    page = 0;
+                  }
+                  for (int ch = 0; ch < L::kChunks; ++ch)
+                    tma_load_3d(dst + ch * L::kChunkBytes + pg * kPageTok * 128, tm,
+                                kv_full(slot), ch * 64, it.hkv, page * kPageTok);
+                }
+              } else {
+                for (int ch = 0; ch < L::kChunks; ++ch) {
+                  if (RAGGED)
+                    tma_load_3d(dst + ch * L::kChunkBytes, tm, kv_full(slot), ch * 64, it.hkv,
+                                it.k_start + j * kBN);
+                  else
+                    tma_load_3d(dst + ch * L::kChunkBytes, tm, kv_full(slot), ch * 64,
+                                j * kBN, kv_z);
+                }
               }
             }
           }
@@ -409,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         int pos = 0, items = 0;
         int tiles[2] = {0, 0};   // S tiles of each query-tile slot in earlier items (phases)
-        ItemWalker<RAGGED> walk;
+        ItemWalker<MODE> walk;
         walk.init(p, cta, C);
         FwdItem it;
         while (ok && walk.next(p, it)) {
@@ -481,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tmem + lane_base + 256 + t * D;
     int tiles = 0, outs = 0;     // S tiles and O tiles of this slot in earlier items (phases)
     bool ok = true;
-    ItemWalker<RAGGED> walk;
+    ItemWalker<MODE> walk;
     walk.init(p, cta, C);
     FwdItem it;
     while (ok && walk.next(p, it)) {
@@ -681,14 +720,16 @@ int encode_3d(CUtensorMap* m, const void* base, bool bf16, int D, int N, int Z) 
   const uint32_t box[3] = {64, 128, 1};
   return encode_tensor_map_16bit(m, base, bf16, 3, dims, strides, box);
 }
-// 3-D map over a packed [T, H, D] tensor (token-major) with a 64 x 1 x 128 box:
-// the same 128 rows of 128 bytes in shared memory as encode_3d's box.
-int encode_packed(CUtensorMap* m, const void* base, bool bf16, int D, int H, int T) {
+// 3-D map over a packed [T, H, D] tensor (token-major) with a 64 x 1 x rows box:
+// rows = 128 lands like encode_3d's box (128 rows of 128 bytes); rows = 16 is one
+// page of a paged pool, eight of which fill the same tile.
+int encode_packed(CUtensorMap* m, const void* base, bool bf16, int D, int H, int T,
+                  int rows = 128) {
   const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(H),
                             static_cast<uint64_t>(T)};
   const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2,
                                static_cast<uint64_t>(H) * static_cast<uint64_t>(D) * 2};
-  const uint32_t box[3] = {64, 1, 128};
+  const uint32_t box[3] = {64, 1, static_cast<uint32_t>(rows)};
   return encode_tensor_map_16bit(m, base, bf16, 3, dims, strides, box);
 }
 
@@ -707,9 +748,11 @@ int fwd_sm_count(int device) {
 
 template <int D, bool BF16>
 int launch_typed(const void* q, const void* k, const void* v, void* o, float* lse,
-                 const int* cu_q, const int* cu_k, int total_q, int total_k, int B, int Hq,
-                 int Hkv, int Nq, int Nk, float scale, int causal, cudaStream_t stream,
-                 int device) {
+                 const FwdLayoutArgs& la, int B, int Hq, int Hkv, int Nq, int Nk, float scale,
+                 int causal, cudaStream_t stream, int device) {
+  const int* cu_q = la.cu_q;
+  const int total_q = la.total_q, total_k = la.total_k;
+  const bool paged = la.block_table != nullptr;
   using L = FwdLayout<D>;
   static bool attr_done[64] = {};
   static std::mutex mu;
@@ -717,11 +760,14 @@ int launch_typed(const void* q, const void* k, const void* v, void* o, float* ls
     std::lock_guard<std::mutex> g(mu);
     if (device < 0 || device >= 64) return set_error(FA_ERR_CUDA, "device ordinal out of range");
     if (!attr_done[device]) {
-      cudaError_t e = cudaFuncSetAttribute(fa_fwd_kernel<D, BF16, false>,
+      cudaError_t e = cudaFuncSetAttribute(fa_fwd_kernel<D, BF16, kDense>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            L::kSmemBytes);
       if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(fa_fwd_kernel<D, BF16, true>,
+        e = cudaFuncSetAttribute(fa_fwd_kernel<D, BF16, kRagged>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(fa_fwd_kernel<D, BF16, kPaged>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
       if (e != cudaSuccess)
         return set_error(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
@@ -735,7 +781,11 @@ int launch_typed(const void* q, const void* k, const void* v, void* o, float* ls
   } else if ((rc = encode_3d(&tq, q, BF16, D, Nq, B * Hq)) != FA_OK) {
     return rc;
   }
-  if (cu_q && total_k > 0) {
+  if (paged) {
+    const int pool_tok = la.num_pages * kPageTok;
+    if ((rc = encode_packed(&tk, k, BF16, D, Hkv, pool_tok, kPageTok)) != FA_OK) return rc;
+    if ((rc = encode_packed(&tv, v, BF16, D, Hkv, pool_tok, kPageTok)) != FA_OK) return rc;
+  } else if (cu_q && total_k > 0) {
     if ((rc = encode_packed(&tk, k, BF16, D, Hkv, total_k)) != FA_OK) return rc;
     if ((rc = encode_packed(&tv, v, BF16, D, Hkv, total_k)) != FA_OK) return rc;
   } else if (!cu_q && Nk > 0) {
@@ -749,9 +799,13 @@ int launch_typed(const void* q, const void* k, const void* v, void* o, float* ls
   prm.o = o;
   prm.lse = lse;
   prm.cu_q = cu_q;
-  prm.cu_k = cu_k;
+  prm.cu_k = la.cu_k;
   prm.total_q = total_q;
   prm.total_k = total_k;
+  prm.block_table = la.block_table;
+  prm.seq_lens_k = la.seq_lens_k;
+  prm.max_pages = la.max_pages;
+  prm.num_pages = la.num_pages;
   prm.B = B;
   prm.Hq = Hq;
   prm.Hkv = Hkv;
@@ -771,12 +825,13 @@ int launch_typed(const void* q, const void* k, const void* v, void* o, float* ls
   if (nsm <= 0) return set_error(FA_ERR_CUDA, "cannot read the SM count of device %d", device);
   const int grid = static_cast<int>(std::min<long long>(items, nsm));
   if (grid == 0) return FA_OK;
-  if (cu_q)
-    fa_fwd_kernel<D, BF16, true><<<static_cast<unsigned>(grid), kThreads, L::kSmemBytes,
-                                   stream>>>(tq, tk, tv, prm);
+  const unsigned g = static_cast<unsigned>(grid);
+  if (paged)
+    fa_fwd_kernel<D, BF16, kPaged><<<g, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, prm);
+  else if (cu_q)
+    fa_fwd_kernel<D, BF16, kRagged><<<g, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, prm);
   else
-    fa_fwd_kernel<D, BF16, false><<<static_cast<unsigned>(grid), kThreads, L::kSmemBytes,
-                                    stream>>>(tq, tk, tv, prm);
+    fa_fwd_kernel<D, BF16, kDense><<<g, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, prm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(FA_ERR_CUDA, "fa_fwd launch: %s", cudaGetErrorString(e));
   return FA_OK;
@@ -785,11 +840,9 @@ int launch_typed(const void* q, const void* k, const void* v, void* o, float* ls
 }  // namespace
 
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
-               const int* cu_q, const int* cu_k, int total_q, int total_k, int B, int Hq,
-               int Hkv, int Nq, int Nk, int D, float scale, int causal, bool bf16,
-               cudaStream_t stream, int device) {
-#define FA_FWD_ARGS q, k, v, o, lse, cu_q, cu_k, total_q, total_k, B, Hq, Hkv, Nq, Nk, scale, \
-                    causal, stream, device
+               const FwdLayoutArgs& la, int B, int Hq, int Hkv, int Nq, int Nk, int D,
+               float scale, int causal, bool bf16, cudaStream_t stream, int device) {
+#define FA_FWD_ARGS q, k, v, o, lse, la, B, Hq, Hkv, Nq, Nk, scale, causal, stream, device
   if (D == 128)
     return bf16 ? launch_typed<128, true>(FA_FWD_ARGS) : launch_typed<128, false>(FA_FWD_ARGS);
   if (D == 64)

@@ -26,13 +26,23 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 // Forward prefill launcher (validated arguments).  bf16 selects bf16 inputs,
 // otherwise fp16.  Returns an FA_* status.
-// cu_q == nullptr: dense [B, H, N, D] tensors; otherwise a ragged batch packed as
-// [total, H, D] with per-sequence row offsets cu_q / cu_k ([B + 1], device) and
-// Nq / Nk bounding the sequence lengths.
+// Batch layout of a forward call.  cu_q == nullptr: dense [B, H, N, D] tensors.
+// Otherwise queries are packed as [total_q, H, D] with per-sequence row offsets
+// cu_q ([B + 1], device) and Nq bounds their lengths; keys/values are either
+// packed the same way (cu_k, total_k; Nk bounds their lengths) or, with
+// block_table != nullptr, held in a page pool [num_pages, 16, Hkv, D] reached
+// through block_table [B, max_pages] with seq_lens_k [B] keys per sequence.
+struct FwdLayoutArgs {
+  const int* cu_q = nullptr;
+  const int* cu_k = nullptr;
+  int total_q = 0, total_k = 0;
+  const int* block_table = nullptr;
+  const int* seq_lens_k = nullptr;
+  int max_pages = 0, num_pages = 0;
+};
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
-               const int* cu_q, const int* cu_k, int total_q, int total_k, int B, int Hq,
-               int Hkv, int Nq, int Nk, int D, float scale, int causal, bool bf16,
-               cudaStream_t stream, int device);
+               const FwdLayoutArgs& la, int B, int Hq, int Hkv, int Nq, int Nk, int D,
+               float scale, int causal, bool bf16, cudaStream_t stream, int device);
 
 // Split-KV paged decode launcher (validated arguments).
 int launch_decode(const void* q, const void* kcache, const void* vcache, const int32_t* block_table,

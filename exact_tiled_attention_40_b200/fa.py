@@ -33,6 +33,8 @@ _SIGS = {
                            _P]),
     "fa_fwd_varlen_fp16": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
                                 _I, _P]),
+    "fa_fwd_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I,
+                          _F, _I, _P]),
     "fa_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _I, _I, _P]),
     "fa_decode_paged_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _I, _I,
                                      _P]),
@@ -142,6 +144,37 @@ def attention_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqle
     lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device) if return_lse else None
     fa_fwd_varlen(q, k, v, o, lse, cu_seqlens_q.contiguous(), cu_seqlens_k.contiguous(), B, Hq,
                   Hkv, int(max_seqlen_q), int(max_seqlen_k), total_q, total_k, D, scale, causal)
+    return o, lse
+
+
+def fa_fwd_paged(q, kcache, vcache, block_table, o, lse, cu_q, seq_lens_k, B, Hq, Hkv, max_q,
+                 max_pages_per_seq, num_pages, total_q, D, page_size, scale, causal, stream=None):
+    """Raw call of the paged-prefill entry point (bf16)."""
+    s = _stream(q.device) if stream is None else ctypes.c_void_p(stream)
+    _check(lib().fa_fwd_paged(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(block_table), _ptr(o),
+                              _ptr(lse), _ptr(cu_q), _ptr(seq_lens_k), B, Hq, Hkv, max_q,
+                              max_pages_per_seq, num_pages, total_q, D, page_size, float(scale),
+                              int(bool(causal)), s), "fa_fwd_paged")
+
+
+def prefill_paged(q, kcache, vcache, block_table, cu_seqlens_q, seq_lens_k, max_seqlen_q,
+                  scale=None, causal=True, return_lse=True):
+    """O [total_q,Hq,D] (and LSE [Hq,total_q]) for packed new queries q [total_q,Hq,D]
+    against a paged bf16 cache [num_pages,16,Hkv,D] (int32 block table and lengths)."""
+    for t in (q, kcache, vcache, block_table, cu_seqlens_q, seq_lens_k):
+        if not t.is_cuda:
+            raise FAError(1, "prefill_paged", "tensors must live on a CUDA device")
+    total_q, Hq, D = q.shape
+    num_pages, page_size, Hkv, _ = kcache.shape
+    B = cu_seqlens_q.numel() - 1
+    if scale is None:
+        scale = D ** -0.5
+    o = torch.empty_like(q)
+    lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device) if return_lse else None
+    fa_fwd_paged(q.contiguous(), kcache, vcache, block_table.contiguous(), o, lse,
+                 cu_seqlens_q.contiguous(), seq_lens_k.contiguous(), B, Hq, Hkv,
+                 int(max_seqlen_q), block_table.shape[1], num_pages, total_q, D, page_size, scale,
+                 causal)
     return o, lse
 
 

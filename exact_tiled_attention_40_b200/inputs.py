@@ -18,6 +18,12 @@ order (so no page is shared); then q ``randn(B, Hq, D)``; then the K pool and
 the V pool, each drawn in chunks of 1024 pages as ``randn(c, page_size, Hkv, D)``.
 Unused block-table entries are 0.
 
+Recipe (paged prefill): one generator seeded with the case seed; key lengths
+``randint(lo, hi + 1, (B,))`` (or listed); query counts listed or equal to the
+key lengths; a permutation of the page pool handed out in sequence order as for
+paged decode; then packed Q [total_q, Hq, D], then the K pool and the V pool
+``randn(num_pages, 16, Hkv, D)``.
+
 Recipe (ragged prefill): one generator seeded with the case seed; the key
 lengths ``randint(lo, hi + 1, (B,))`` unless the case lists them; query lengths
 equal to the key lengths (or listed); then packed Q [total_q, Hq, D], K and V
@@ -31,7 +37,9 @@ from dataclasses import dataclass, field
 import torch
 
 __all__ = ["PrefillCase", "DecodeCase", "VarlenCase", "PREFILL_CASES", "DECODE_CASES",
-           "VARLEN_CASES", "make_prefill", "make_decode", "make_varlen", "varlen_flops",
+           "VARLEN_CASES", "PagedPrefillCase", "PAGED_PREFILL_CASES", "make_paged_prefill",
+           "make_prefill",
+           "make_decode", "make_varlen", "varlen_flops",
            "sample_rows"]
 
 _DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16}
@@ -257,4 +265,66 @@ VARLEN_CASES = {
     # a serving-like mix: 16 sequences, lengths U[256, 8192], Llama-3-8B heads, causal
     "varlen_b16_hq32_hkv8_d128_causal": VarlenCase("varlen_b16_hq32_hkv8_d128_causal", 16, 32, 8,
                                                     128, "bf16", True, seed=5, lo=256, hi=8192),
+}
+
+
+@dataclass(frozen=True)
+class PagedPrefillCase:
+    """New queries of B sequences against their keys/values in a 16-token page
+    pool: sequence b has nk[b] cached keys and its last nq[b] tokens query them."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    D: int
+    causal: bool
+    seed: int
+    num_pages: int
+    lo: int = 1
+    hi: int = 1
+    nq: tuple = ()
+    nk: tuple = ()
+    page_size: int = 16
+
+    @property
+    def softmax_scale(self) -> float:
+        return 1.0 / math.sqrt(self.D)
+
+
+def make_paged_prefill(case: PagedPrefillCase):
+    """q [total_q, Hq, D], kcache, vcache [num_pages, 16, Hkv, D] (bf16), block_table
+    [B, max_pages], cu_q [B + 1] and seq_lens_k [B] (int32), all on the CPU."""
+    gen = torch.Generator("cpu").manual_seed(case.seed)
+    if case.nk:
+        nk = torch.tensor(case.nk, dtype=torch.int64)
+    else:
+        nk = torch.randint(case.lo, case.hi + 1, (case.B,), generator=gen)
+    nq = torch.tensor(case.nq, dtype=torch.int64) if case.nq else nk.clone()
+    npages = [(int(n) + case.page_size - 1) // case.page_size for n in nk]
+    max_pages = max(1, max(npages))
+    if sum(npages) > case.num_pages:
+        raise ValueError("page pool too small for the drawn lengths")
+    perm = torch.randperm(case.num_pages, generator=gen)
+    table = torch.zeros(case.B, max_pages, dtype=torch.int32)
+    used = 0
+    for b, n in enumerate(npages):
+        table[b, :n] = perm[used:used + n].to(torch.int32)
+        used += n
+    cu_q = torch.zeros(case.B + 1, dtype=torch.int32)
+    cu_q[1:] = torch.cumsum(nq, 0).to(torch.int32)
+    q = torch.randn(int(cu_q[-1]), case.Hq, case.D, generator=gen).to(torch.bfloat16)
+    shape = (case.num_pages, case.page_size, case.Hkv, case.D)
+    kc = torch.randn(shape, generator=gen).to(torch.bfloat16)
+    vc = torch.randn(shape, generator=gen).to(torch.bfloat16)
+    return q, kc, vc, table, cu_q, nk.to(torch.int32)
+
+
+PAGED_PREFILL_CASES = {
+    # chunked prefill: 16 sequences with 1024-8192 cached tokens each; the last
+    # 512 tokens of every sequence are the new queries (causal), Llama-3-8B heads
+    "paged_prefill_b16_chunk512_hq32_hkv8_d128": PagedPrefillCase(
+        "paged_prefill_b16_chunk512_hq32_hkv8_d128", 16, 32, 8, 128, True, seed=6,
+        num_pages=16 * 512, nq=(512,) * 16,
+        nk=(1024, 8192, 2048, 4096, 3000, 6000, 5120, 1536, 7000, 2500, 4500, 8000, 1800, 3500,
+            6500, 5000)),
 }

@@ -17,14 +17,15 @@ import statistics
 import torch
 
 from . import fa
-from .inputs import (DECODE_CASES, PREFILL_CASES, VARLEN_CASES, make_decode, make_prefill,
-                     make_varlen, varlen_flops)
+from .inputs import (DECODE_CASES, PAGED_PREFILL_CASES, PREFILL_CASES, VARLEN_CASES,
+                     make_decode, make_paged_prefill, make_prefill, make_varlen, varlen_flops)
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--case", required=True,
-                    choices=sorted(PREFILL_CASES) + sorted(DECODE_CASES) + sorted(VARLEN_CASES))
+                    choices=sorted(PREFILL_CASES) + sorted(DECODE_CASES) + sorted(VARLEN_CASES)
+                    + sorted(PAGED_PREFILL_CASES))
     ap.add_argument("--iters", type=int, default=5)
     args = ap.parse_args()
     dev = torch.device("cuda", 0)
@@ -41,6 +42,22 @@ def main():
             fa.fa_fwd(q, k, v, o, lse, c.B, c.Hq, c.Hkv, c.Nq, c.Nk, c.D, c.softmax_scale,
                       c.causal, stream=stream.cuda_stream)
         work, unit = c.flops / 1e12, "TFLOP/s"
+    elif args.case in PAGED_PREFILL_CASES:
+        c = PAGED_PREFILL_CASES[args.case]
+        q, kc, vc, table, cu_q, lens = make_paged_prefill(c)
+        cu_k = torch.zeros_like(cu_q)
+        cu_k[1:] = torch.cumsum(lens, 0)
+        flops = varlen_flops(cu_q, cu_k, c.Hq, c.D, c.causal)
+        max_q = int((cu_q[1:] - cu_q[:-1]).max())
+        q, kc, vc, table, cu_q, lens = (t.to(dev) for t in (q, kc, vc, table, cu_q, lens))
+        o = torch.empty_like(q)
+        lse = torch.empty((c.Hq, q.shape[0]), dtype=torch.float32, device=dev)
+
+        def launch():
+            fa.fa_fwd_paged(q, kc, vc, table, o, lse, cu_q, lens, c.B, c.Hq, c.Hkv, max_q,
+                            table.shape[1], c.num_pages, q.shape[0], c.D, c.page_size,
+                            c.softmax_scale, c.causal, stream=stream.cuda_stream)
+        work, unit = flops / 1e12, "TFLOP/s"
     elif args.case in VARLEN_CASES:
         c = VARLEN_CASES[args.case]
         q, k, v, cu_q, cu_k = make_varlen(c)

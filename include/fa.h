@@ -111,6 +111,32 @@ int fa_fwd_varlen_fp16(const void* q, const void* k, const void* v, void* o, flo
                        int D, float scale, int causal, fa_stream_t stream);
 
 /*
+ * Prefill against a paged KV cache (bf16): the new query tokens of each
+ * sequence attend over that sequence's keys and values held in the page pool
+ * (cabseo.com "Advanced techniques for enhancing LLM throughput", section
+ * "Paged attention"), e.g. a prompt prefilled in chunks after earlier chunks
+ * were written to the cache.
+ *   q            [total_q, Hq, D] bf16, sequence b's queries are rows
+ *                [cu_seqlens_q[b], cu_seqlens_q[b+1]) (int32 [B + 1] on the device)
+ *   kcache/vcache [num_pages, page_size, Hkv, D] bf16, as for fa_decode_paged
+ *   block_table  [B, max_pages_per_seq] int32, seq_lens_k [B] int32: sequence b
+ *                has seq_lens_k[b] keys, token t in page block_table[b][t / 16]
+ *   o            [total_q, Hq, D] bf16 (written rows of valid sequences only)
+ *   lse          [Hq, total_q] fp32 (written; may be NULL)
+ * causal: the queries are the last Nq_b tokens of the sequence (bottom-right
+ * alignment); needs Nq_b <= seq_lens_k[b].  Supported: page_size == 16, D 64 or
+ * 128, GQA as for fa_fwd.  Lengths and offsets breaking these rules skip the
+ * sequence and raise FA_ERR_DEVICE_INDEX; a block-table entry outside
+ * [0, num_pages) is read as page 0 and raises the same status.  No workspace is
+ * allocated.
+ */
+int fa_fwd_paged(const void* q, const void* kcache, const void* vcache,
+                 const int32_t* block_table, void* o, float* lse, const int32_t* cu_seqlens_q,
+                 const int32_t* seq_lens_k, int B, int Hq, int Hkv, int max_seqlen_q,
+                 int max_pages_per_seq, int num_pages, int total_q, int D, int page_size,
+                 float scale, int causal, fa_stream_t stream);
+
+/*
  * Decode over a paged KV cache: one new query token per sequence attends over
  * all of that sequence's cached keys and values (no mask beyond its length).
  *   q           [B, Hq, D] bf16
