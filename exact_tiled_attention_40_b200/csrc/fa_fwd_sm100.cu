@@ -56,18 +56,24 @@ constexpr uint32_t kRegsControl = 72;    // warps 8-11
 constexpr uint32_t kRegsSoftmax = 216;   // warps 0-7
 static_assert(kRegsControl * 128 + kRegsSoftmax * 256 <= 384 * 168, "register split");
 
-template <int D>
+constexpr int kSchedMax = 2048;   // entries of the work-sorted list of ragged batches
+
+// SCHED: the ragged and paged kernels also keep their work-sorted (pair,
+// sequence) list in shared memory, and give up one K/V slot at D = 128 for it.
+template <int D, bool SCHED = false>
 struct FwdLayout {
   static constexpr int kChunks = D / 64;              // 128-byte swizzle atoms along D
   static constexpr int kChunkBytes = kBM * 128;       // one atom column of a 128-row tile
   static constexpr int kTileBytes = kBM * D * 2;      // a 128-row tile of Q, K or V
-  static constexpr int kSlots = D == 128 ? 5 : 8;     // K/V ring slots
+  static constexpr int kSlots = D == 128 ? (SCHED ? 4 : 5) : 8;   // K/V ring slots
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
   static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 4 + 2 + 1 + 1;
-  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + slack for 1024-byte alignment
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;   // tmem address, abort, list size, ok
+  static constexpr int kSchedOff = kMiscOff + 16;
+  static constexpr int kSmemBytes =
+      kSchedOff + (SCHED ? kSchedMax * 4 : 0) + 1024;     // + slack for 1024-byte alignment
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -175,18 +181,29 @@ __device__ __forceinline__ FwdItem make_item(const FwdParams& p, int b, int h, i
 // Ragged batches list only pairs that start inside their sequence (pair m of
 // sequence b for m < ceil(Nq_b / 256)), so the rounds contain no empty items;
 // every role of the CTA walks a cursor along that list, whose indices only grow.
-// (Separate instantiations keep the dense kernel free of the cursor.)
+// When the list is small enough (<= 2048 (pair, sequence) entries, B <= 1024,
+// pairs <= 1024, <= 4095 key tiles) the CTA first sorts it by each entry's key
+// tiles, heaviest first, in shared memory, so that the snake rounds balance
+// sequences of very different lengths too.  (Separate instantiations keep the
+// dense kernel free of all this.)
 template <int MODE>
 struct ItemWalker {
   int cta, C, r, total;
   int idx, m, b, h;   // ragged cursor: list entry idx is (pair m, sequence b, head h)
+  const uint32_t* sorted;   // ragged: work-sorted (pair, sequence) keys, or null
 
-  __device__ void init(const FwdParams& p, int cta_, int C_) {
+  __device__ void init(const FwdParams& p, int cta_, int C_, const uint32_t* sorted_ = nullptr,
+                       int n_sorted = 0) {
     cta = cta_;
     C = C_;
     r = 0;
+    sorted = sorted_;
     if constexpr (MODE == kDense) {
       total = p.num_items;
+      return;
+    }
+    if (sorted) {
+      total = n_sorted * p.Hq;
       return;
     }
     int sum = 0, pmax = 0;
@@ -230,6 +247,13 @@ struct ItemWalker {
     ++r;
     if (i >= total) return false;
     if constexpr (MODE != kDense) {
+      if (sorted) {
+        const int e = i / p.Hq;
+        const uint32_t key = sorted[e];
+        it = make_item<MODE>(p, static_cast<int>(key & 1023u),
+                             i - e * p.Hq, 1023 - static_cast<int>((key >> 10) & 1023u));
+        return true;
+      }
       advance(p, i);
       it = make_item<MODE>(p, b, h, m);
     } else {
@@ -248,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   constexpr bool RAGGED = MODE != kDense;
-  using L = FwdLayout<D>;
+  using L = FwdLayout<D, RAGGED>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -309,6 +333,64 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Ragged batches: the (pair, sequence) entries in shared memory, sorted by key
+  // (4095 - key tiles) << 20 | (1023 - pair) << 10 | sequence, ascending.
+  const uint32_t* sorted = nullptr;
+  int n_sorted = 0;
+  if constexpr (RAGGED) {
+    uint32_t* list = reinterpret_cast<uint32_t*>(smem + L::kSchedOff);
+    int* list_n = reinterpret_cast<int*>(smem + L::kMiscOff + 8);
+    volatile int* list_ok = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 12);
+    if (tid == 0) {
+      *list_n = 0;
+      *list_ok = p.B <= 1024 ? 1 : 0;
+    }
+    __syncthreads();
+    if (*list_ok) {
+      for (int bb = tid; bb < p.B; bb += kThreads) {
+        int q0, nq, k0, nk;
+        if (!ragged_rows<MODE>(p, bb, q0, nq, k0, nk)) continue;
+        const int pairs = (nq + 2 * kBM - 1) / (2 * kBM);
+        for (int m = 0; m < pairs; ++m) {
+          const int w = max(kv_tiles_for(m * 2 * kBM, nq, nk, p.causal),
+                            kv_tiles_for(m * 2 * kBM + kBM, nq, nk, p.causal));
+          const int at = atomicAdd(list_n, 1);
+          if (at < kSchedMax && m < 1024 && w < 4096)
+            list[at] = (static_cast<uint32_t>(4095 - w) << 20) |
+                       (static_cast<uint32_t>(1023 - m) << 10) | static_cast<uint32_t>(bb);
+          else
+            *list_ok = 0;
+        }
+      }
+    }
+    __syncthreads();
+    if (*list_ok) {
+      // the keys are distinct, so the sorted order does not depend on the order
+      // in which the threads appended them: bitonic sort, padded to a power of 2
+      const int E = *list_n;
+      int N = 1;
+      while (N < E) N <<= 1;
+      for (int i = E + tid; i < N; i += kThreads) list[i] = 0xffffffffu;
+      __syncthreads();
+      for (int k = 2; k <= N; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+          for (int i = tid; i < N; i += kThreads) {
+            const int ixj = i ^ j;
+            if (ixj > i) {
+              const uint32_t a = list[i], c2 = list[ixj];
+              if ((a > c2) == ((i & k) == 0)) {
+                list[i] = c2;
+                list[ixj] = a;
+              }
+            }
+          }
+          __syncthreads();
+        }
+      }
+      sorted = list;
+      n_sorted = E;
+    }
+  }
   if (warp >= 8) {
     regs_dec<kRegsControl>();
     if (warp == 8) {
@@ -322,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int pos = 0, items = 0;
         bool ok = true;
         ItemWalker<MODE> walk;
-        walk.init(p, cta, C);
+        walk.init(p, cta, C, sorted, n_sorted);
         FwdItem it;
         while (ok && walk.next(p, it)) {
           const int n_max = max(it.n0, it.n1);
@@ -449,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int pos = 0, items = 0;
         int tiles[2] = {0, 0};   // S tiles of each query-tile slot in earlier items (phases)
         ItemWalker<MODE> walk;
-        walk.init(p, cta, C);
+        walk.init(p, cta, C, sorted, n_sorted);
         FwdItem it;
         while (ok && walk.next(p, it)) {
           const int n_max = max(it.n0, it.n1);
@@ -521,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int tiles = 0, outs = 0;     // S tiles and O tiles of this slot in earlier items (phases)
     bool ok = true;
     ItemWalker<MODE> walk;
-    walk.init(p, cta, C);
+    walk.init(p, cta, C, sorted, n_sorted);
     FwdItem it;
     while (ok && walk.next(p, it)) {
     const int q_row0 = it.q_row0;
@@ -753,7 +835,8 @@ int launch_typed(const void* q, const void* k, const void* v, void* o, float* ls
   const int* cu_q = la.cu_q;
   const int total_q = la.total_q, total_k = la.total_k;
   const bool paged = la.block_table != nullptr;
-  using L = FwdLayout<D>;
+  using L = FwdLayout<D, false>;
+  using LR = FwdLayout<D, true>;   // ragged and paged batches
   static bool attr_done[64] = {};
   static std::mutex mu;
   {
@@ -765,10 +848,10 @@ int launch_typed(const void* q, const void* k, const void* v, void* o, float* ls
                                            L::kSmemBytes);
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(fa_fwd_kernel<D, BF16, kRagged>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, LR::kSmemBytes);
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(fa_fwd_kernel<D, BF16, kPaged>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, LR::kSmemBytes);
       if (e != cudaSuccess)
         return set_error(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
       attr_done[device] = true;
@@ -827,9 +910,9 @@ int launch_typed(const void* q, const void* k, const void* v, void* o, float* ls
   if (grid == 0) return FA_OK;
   const unsigned g = static_cast<unsigned>(grid);
   if (paged)
-    fa_fwd_kernel<D, BF16, kPaged><<<g, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, prm);
+    fa_fwd_kernel<D, BF16, kPaged><<<g, kThreads, LR::kSmemBytes, stream>>>(tq, tk, tv, prm);
   else if (cu_q)
-    fa_fwd_kernel<D, BF16, kRagged><<<g, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, prm);
+    fa_fwd_kernel<D, BF16, kRagged><<<g, kThreads, LR::kSmemBytes, stream>>>(tq, tk, tv, prm);
   else
     fa_fwd_kernel<D, BF16, kDense><<<g, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, prm);
   cudaError_t e = cudaGetLastError();
