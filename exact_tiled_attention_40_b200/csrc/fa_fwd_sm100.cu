@@ -6,13 +6,19 @@
 // with the softmax decomposition and merge of section "The Mathematics of
 // Flash Attention".  O is kept unnormalised and divided by L once at the end.
 //
-// One CTA owns two 128-row query tiles (Q0, Q1) of one (batch, head) and streams
-// the 128-key K/V tiles of the matching KV head (GQA, devhandbook example 5)
-// through a ring of shared-memory slots.  Warp roles (384 threads, 3 warpgroups):
+// Persistent: one CTA per SM walks a list of work items, each two 128-row query
+// tiles (Q0, Q1) of one (sequence, head), streaming the 128-key K/V tiles of the
+// matching KV head (GQA, devhandbook example 5) through a ring of shared-memory
+// slots whose positions, like every barrier's phase, run on across items.
+// Three instantiations share this code: dense [B, H, N, D] tensors, ragged
+// batches packed as [total, H, D] with device row offsets, and ragged queries
+// against keys/values in a 16-token page pool reached through a block table.
+// Warp roles (384 threads, 3 warpgroups):
 //   warps 0-3   softmax warpgroup for Q0   (thread r owns query row r = TMEM lane r)
 //   warps 4-7   softmax warpgroup for Q1
-//   warp  8     TMA producer: Q tiles once, then K_j, V_j into the slot ring
-//   warp  9     TMEM allocator and single-thread tcgen05 MMA issuer
+//   warp  8     TMA producer: per item the Q tiles, then K_j, V_j into the slot ring
+//   warp  9     TMEM allocator and MMA issuer (the warp runs the loop, one elected
+//               lane issues the tcgen05 MMAs and commits)
 //   warps 10-11 idle
 // The control warpgroup (warps 8-11) hands registers to the softmax warpgroups
 // (setmaxnreg): 72 and 216 per-thread registers over 128 + 256 threads equal

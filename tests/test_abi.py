@@ -109,3 +109,31 @@ def test_varlen_empty_batch_is_a_noop(lib):
     assert varlen(lib, tq=0) == 0
     assert varlen(lib, max_q=0) == 0
     assert varlen(lib, tk=0, k=None, v=None, q=FAKE) in (0, E["FA_ERR_NO_DEVICE"])
+
+
+def paged(lib, B=2, Hq=4, Hkv=2, max_q=9, maxp=4, npages=10, tq=12, D=128, page=16, scale=0.1,
+          causal=1, q=FAKE, kc=FAKE, vc=FAKE, table=FAKE, o=FAKE, cuq=FAKE, lens=FAKE):
+    return lib.fa_fwd_paged(q, kc, vc, table, o, None, cuq, lens, B, Hq, Hkv, max_q, maxp, npages,
+                            tq, D, page, scale, causal, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=-1), "FA_ERR_INVALID_ARG"),
+    (dict(D=96), "FA_ERR_UNSUPPORTED"),
+    (dict(page=32), "FA_ERR_UNSUPPORTED"),
+    (dict(Hq=3), "FA_ERR_INVALID_ARG"),
+    (dict(maxp=0), "FA_ERR_INVALID_ARG"),
+    (dict(npages=0), "FA_ERR_INVALID_ARG"),
+    (dict(table=None), "FA_ERR_INVALID_ARG"),
+    (dict(lens=None), "FA_ERR_INVALID_ARG"),
+    (dict(kc=FAKE + 4), "FA_ERR_INVALID_ARG"),
+    (dict(scale=float("inf")), "FA_ERR_INVALID_ARG"),
+])
+def test_paged_prefill_rejects_bad_arguments_on_the_host(lib, kw, code):
+    assert paged(lib, **kw) == E[code]
+    assert lib.fa_last_error_string()
+
+
+def test_paged_prefill_empty_batch_is_a_noop(lib):
+    assert paged(lib, B=0) == 0
+    assert paged(lib, tq=0) == 0
