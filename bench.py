@@ -31,17 +31,21 @@ import subprocess
 import sys
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from exact_tiled_attention_40_b200.inputs import (DECODE_CASES, PREFILL_CASES,  # noqa: E402
-                                                  make_decode, make_prefill)
+from exact_tiled_attention_40_b200.inputs import (  # noqa: E402
+    DECODE_CASES, PAGED_PREFILL_CASES, PREFILL_CASES, VARLEN_CASES, make_decode,
+    make_paged_prefill, make_prefill, make_varlen, varlen_flops)
 
 METRIC = "attention TFLOP/s & % BF16 tensor peak (prefill); decode KV GB/s & % HBM peak"
 PREFILL = PREFILL_CASES["gqa_b1_hq32_hkv8_n8192_d128_causal"]
 DECODE = DECODE_CASES["decode_b64_hq32_hkv8_d128_page16"]
+RAGGED = VARLEN_CASES["varlen_b16_hq32_hkv8_d128_causal"]
+PAGED = PAGED_PREFILL_CASES["paged_prefill_b16_chunk512_hq32_hkv8_d128"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 256 << 20
 
@@ -184,6 +188,123 @@ def oracle_decode_sample(seqs: int = 8):
     dt = time.perf_counter() - t0
     kv_bytes = int(lens[:seqs].sum()) * DECODE.Hkv * DECODE.D * 2 * 2
     return kv_bytes / dt / 1e9, dt, f"{seqs} of {DECODE.B} sequences of {DECODE.name}, fp64"
+
+
+def oracle_ragged_sample(heads: int = 4):
+    """fp64 ragged-batch oracle on the shortest sequence of the ragged workload,
+    its first `heads` query heads.  Returns (TFLOP/s, seconds, sample text)."""
+    import oracle
+    q, k, v, cu_q, cu_k = make_varlen(RAGGED)
+    nq = cu_q[1:] - cu_q[:-1]
+    b = int(torch.argmin(nq))
+    q0, q1, k0, k1 = (int(x) for x in (cu_q[b], cu_q[b + 1], cu_k[b], cu_k[b + 1]))
+    g = RAGGED.Hq // RAGGED.Hkv
+    hk = max(1, heads // g)
+    qs = q[q0:q1, :heads].float().double().numpy()
+    ks = k[k0:k1, :hk].float().double().numpy()
+    vs = v[k0:k1, :hk].float().double().numpy()
+    cu1 = np.array([0, q1 - q0])
+    ck1 = np.array([0, k1 - k0])
+    t0 = time.perf_counter()
+    oracle.varlen_attention(qs, ks, vs, cu1, ck1, RAGGED.softmax_scale, RAGGED.causal)
+    dt = time.perf_counter() - t0
+    flops = varlen_flops(torch.tensor(cu1), torch.tensor(ck1), heads, RAGGED.D, RAGGED.causal)
+    return flops / dt / 1e12, dt, (f"sequence {b} ({q1 - q0} tokens), {heads} of {RAGGED.Hq} "
+                                   f"query heads of {RAGGED.name}, fp64")
+
+
+def oracle_paged_sample(heads: int = 4):
+    """fp64 paged-prefill oracle on the sequence with the fewest cached keys of the
+    paged workload, its first `heads` query heads.  Returns (TFLOP/s, seconds, text)."""
+    import oracle
+    q, kc, vc, table, cu_q, lens = make_paged_prefill(PAGED)
+    b = int(torch.argmin(lens))
+    q0, q1 = int(cu_q[b]), int(cu_q[b + 1])
+    g = PAGED.Hq // PAGED.Hkv
+    hk = max(1, heads // g)
+    qs = q[q0:q1, :heads].float().double().numpy()
+    kcs = kc[:, :, :hk].float().numpy()
+    vcs = vc[:, :, :hk].float().numpy()
+    cu1 = np.array([0, q1 - q0])
+    t0 = time.perf_counter()
+    oracle.paged_prefill(qs, kcs, vcs, table[b:b + 1].numpy(), cu1, lens[b:b + 1].numpy(),
+                         PAGED.softmax_scale, PAGED.causal, PAGED.page_size)
+    dt = time.perf_counter() - t0
+    ck1 = torch.tensor([0, int(lens[b])])
+    flops = varlen_flops(torch.tensor(cu1), ck1, heads, PAGED.D, PAGED.causal)
+    return flops / dt / 1e12, dt, (f"sequence {b} ({q1 - q0} queries, {int(lens[b])} keys), "
+                                   f"{heads} of {PAGED.Hq} query heads of {PAGED.name}, fp64")
+
+
+def widened_rows(fa, dev, stream, flush, warmup, steps, peaks, peak_src):
+    """Ragged and paged prefill (rows added beyond the headline path), each timed
+    like the headline kernels with its roofline fraction and an oracle sample.
+    A failure here is reported in the row and does not touch the headline."""
+    out = {}
+    sp = stream.cuda_stream
+
+    def timed(launch):
+        ts = []
+        for i in range(warmup + steps):
+            flush.fill_(i & 0xff)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            launch()
+            b.record(stream)
+            b.synchronize()
+            if i >= warmup:
+                ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    def row(name, flops, ms, sample_fn):
+        tf = flops / (ms * 1e-3) / 1e12
+        otf, odt, sample = sample_fn()
+        return {"workload": name, "value": tf, "unit": "TFLOP/s", "ms_per_launch": ms,
+                "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"],
+                             "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"],
+                             "peak_source": f"{peak_src} burst bf16"},
+                "cpu_baseline": {"value": otf, "unit": "TFLOP/s", "cores": cpu_threads(),
+                                 "kind": "oracle", "sample": sample, "seconds": odt}}
+
+    try:
+        c = RAGGED
+        q_h, k_h, v_h, cq_h, ck_h = make_varlen(c)
+        flops = varlen_flops(cq_h, ck_h, c.Hq, c.D, c.causal)
+        max_q = int((cq_h[1:] - cq_h[:-1]).max())
+        max_k = int((ck_h[1:] - ck_h[:-1]).max())
+        q, k, v, cq, ck = (t.to(dev) for t in (q_h, k_h, v_h, cq_h, ck_h))
+        o = torch.empty_like(q)
+        lse = torch.empty((c.Hq, q.shape[0]), dtype=torch.float32, device=dev)
+        ms = timed(lambda: fa.fa_fwd_varlen(q, k, v, o, lse, cq, ck, c.B, c.Hq, c.Hkv, max_q,
+                                            max_k, q.shape[0], k.shape[0], c.D, c.softmax_scale,
+                                            c.causal, stream=sp))
+        if fa.device_status() != 0:
+            raise RuntimeError(fa.last_error())
+        out["ragged_prefill"] = row(c.name, flops, ms, oracle_ragged_sample)
+        del q, k, v, o, lse
+    except Exception as e:  # reported, never fatal for the headline line
+        out["ragged_prefill"] = {"workload": RAGGED.name, "error": f"{type(e).__name__}: {e}"[:300]}
+    try:
+        c = PAGED
+        q_h, kc_h, vc_h, t_h, cq_h, l_h = make_paged_prefill(c)
+        ck_h = torch.zeros_like(cq_h)
+        ck_h[1:] = torch.cumsum(l_h, 0)
+        flops = varlen_flops(cq_h, ck_h, c.Hq, c.D, c.causal)
+        max_q = int((cq_h[1:] - cq_h[:-1]).max())
+        q, kc, vc, tab, cq, ln = (t.to(dev) for t in (q_h, kc_h, vc_h, t_h, cq_h, l_h))
+        o = torch.empty_like(q)
+        lse = torch.empty((c.Hq, q.shape[0]), dtype=torch.float32, device=dev)
+        ms = timed(lambda: fa.fa_fwd_paged(q, kc, vc, tab, o, lse, cq, ln, c.B, c.Hq, c.Hkv, max_q,
+                                           tab.shape[1], c.num_pages, q.shape[0], c.D,
+                                           c.page_size, c.softmax_scale, c.causal, stream=sp))
+        if fa.device_status() != 0:
+            raise RuntimeError(fa.last_error())
+        out["paged_prefill"] = row(c.name, flops, ms, oracle_paged_sample)
+        del q, kc, vc, o, lse
+    except Exception as e:  # reported, never fatal for the headline line
+        out["paged_prefill"] = {"workload": PAGED.name, "error": f"{type(e).__name__}: {e}"[:300]}
+    return out
 
 
 def run_reference(args, world, rank):
@@ -380,6 +501,9 @@ def main():
         tf, dt, sample = oracle_prefill_sample(heads=8)
         line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cpu_threads(),
                                 "kind": "oracle", "sample": sample, "seconds": dt}
+        # rows beyond the headline path, measured outside its timed region
+        line["widened"] = widened_rows(fa, dev, stream, flush, args.warmup, min(args.steps, 10),
+                                       peaks, peak_src)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if pg is not None:
