@@ -5,6 +5,7 @@ import this package.  The library never does.
 """
 from .attention_fp64 import (  # noqa: F401
     attention,
+    attention_backward,
     attention_rows,
     blockwise_attention,
     causal_allowed,

@@ -359,3 +359,44 @@ def paged_prefill(q, kcache, vcache, block_table, cu_seqlens_q, seq_lens_k, scal
         O[q0:q1] = np.transpose(o[0], (1, 0, 2))
         LSE[:, q0:q1] = lse[0]
     return O, LSE
+
+
+def attention_backward(q, k, v, o, lse, do, scale: float, causal: bool):
+    """Gradients of the attention output with respect to Q, K and V.
+
+    [unite] section "Core Concepts", recomputation: instead of storing the
+    attention matrix, the backward pass recomputes what it needs.  Reading: the
+    probabilities are rebuilt from the saved row LSE as P = exp(scale * Q K^T -
+    LSE) (masked entries 0), then the chain rule through O = P V and the row
+    softmax gives
+        dV = P^T dO,  dP = dO V^T,  dS = P * (dP - rowsum(dO * O)),
+        dQ = scale * dS K,  dK = scale * dS^T Q,
+    with dK, dV of a KV head summed over the query heads that share it (GQA).
+    q, o, do [B, Hq, Nq, D]; k, v [B, Hkv, Nk, D]; lse [B, Hq, Nq] (natural log).
+    Returns dQ, dK, dV in float64 with the shapes of q, k, v.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    o = np.asarray(o, dtype=np.float64)
+    do = np.asarray(do, dtype=np.float64)
+    lse = np.asarray(lse, dtype=np.float64)
+    B, Hq, Hkv, Nq, Nk, D = _check_shapes(q, k, v)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    allowed = causal_allowed(Nq, Nk) if causal else np.ones((Nq, Nk), dtype=bool)
+    for b in range(B):
+        for h in range(Hq):
+            g = kv_head_of(h, Hq, Hkv)
+            s = scale * (q[b, h] @ k[b, g].T)
+            finite = np.isfinite(lse[b, h])[:, None]
+            p = np.where(allowed & finite, np.exp(s - np.where(finite, lse[b, h][:, None], 0.0)),
+                         0.0)
+            dv[b, g] += p.T @ do[b, h]
+            dp = do[b, h] @ v[b, g].T
+            delta = np.sum(do[b, h] * o[b, h], axis=1, keepdims=True)
+            ds = p * (dp - delta)
+            dq[b, h] = scale * (ds @ k[b, g])
+            dk[b, g] += scale * (ds.T @ q[b, h])
+    return dq, dk, dv

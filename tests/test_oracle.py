@@ -383,3 +383,63 @@ def test_paged_prefill_equals_contiguous_ragged_attention():
         O_ref, L_ref = _padded_library(q, k, v, cu_q, cu_k, 0.5, causal)
         np.testing.assert_allclose(O, O_ref, atol=TIGHT)
         np.testing.assert_allclose(L, L_ref, atol=TIGHT)
+
+
+# ---------------------------------------------------------------- backward (recomputation)
+@pytest.mark.parametrize("Hq,Hkv,Nq,Nk,causal", [(2, 2, 7, 7, False), (4, 2, 5, 9, True),
+                                                   (4, 1, 6, 6, True)])
+def test_backward_matches_float64_library_autograd(Hq, Hkv, Nq, Nk, causal):
+    """dQ, dK, dV against torch autograd through float64 library attention
+    (explicit bottom-right mask, K/V heads repeated for GQA)."""
+    q, k, v = rand((2, Hq, Nq, 8), 130), rand((2, Hkv, Nk, 8), 131), rand((2, Hkv, Nk, 8), 132)
+    do = rand((2, Hq, Nq, 8), 133)
+    O, L = oracle.attention(q, k, v, 0.4, causal)
+    dq, dk, dv = oracle.attention_backward(q, k, v, O, L, do, 0.4, causal)
+    tq, tk, tv = (torch.from_numpy(x).requires_grad_(True) for x in (q, k, v))
+    rep = Hq // Hkv
+    mask = torch.ones(Nq, Nk, dtype=torch.bool).tril(diagonal=Nk - Nq) if causal else None
+    o = torch.nn.functional.scaled_dot_product_attention(
+        tq, tk.repeat_interleave(rep, dim=1), tv.repeat_interleave(rep, dim=1), attn_mask=mask,
+        scale=0.4)
+    o.backward(torch.from_numpy(do))
+    np.testing.assert_allclose(dq, tq.grad.numpy(), atol=1e-10)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), atol=1e-10)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), atol=1e-10)
+
+
+def test_backward_matches_finite_differences():
+    """Central differences of <dO, O(Q, K, V)> on a tiny causal GQA case."""
+    q, k, v = rand((1, 2, 3, 4), 134), rand((1, 1, 4, 4), 135), rand((1, 1, 4, 4), 136)
+    do = rand((1, 2, 3, 4), 137)
+    O, L = oracle.attention(q, k, v, 0.7, True)
+    grads = oracle.attention_backward(q, k, v, O, L, do, 0.7, True)
+    eps = 1e-6
+    for which, g in zip(range(3), grads):
+        base = [q, k, v]
+        x = base[which]
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = list(base)
+            args_m = list(base)
+            args_p[which] = xp
+            args_m[which] = xm
+            fp = np.sum(do * oracle.attention(*args_p, 0.7, True)[0])
+            fm = np.sum(do * oracle.attention(*args_m, 0.7, True)[0])
+            num[idx] = (fp - fm) / (2 * eps)
+        np.testing.assert_allclose(g, num, atol=1e-7)
+
+
+def test_pins_catch_a_missing_delta_term():
+    """Dropping the rowsum(dO * O) term (a plausible slip) fails the library check."""
+    q, k, v = rand((1, 1, 5, 4), 138), rand((1, 1, 5, 4), 139), rand((1, 1, 5, 4), 140)
+    do = rand((1, 1, 5, 4), 141)
+    O, L = oracle.attention(q, k, v, 0.5, False)
+    dq_bad, _, _ = oracle.attention_backward(q, k, v, np.zeros_like(O), L, do, 0.5, False)
+    tq = torch.from_numpy(q).requires_grad_(True)
+    o = torch.nn.functional.scaled_dot_product_attention(tq, torch.from_numpy(k),
+                                                         torch.from_numpy(v), scale=0.5)
+    o.backward(torch.from_numpy(do))
+    assert np.max(np.abs(dq_bad - tq.grad.numpy())) > 1e-3
