@@ -24,6 +24,10 @@ key lengths; a permutation of the page pool handed out in sequence order as for
 paged decode; then packed Q [total_q, Hq, D], then the K pool and the V pool
 ``randn(num_pages, 16, Hkv, D)``.
 
+Recipe (FP8 forward): the bf16 inputs of the named prefill case, drawn as
+above; the rotation's D signs from their own generator seeded with the case's
+sign seed, ``rand(D) < 0.5`` giving -1.
+
 Recipe (ragged prefill): one generator seeded with the case seed; the key
 lengths ``randint(lo, hi + 1, (B,))`` unless the case lists them; query lengths
 equal to the key lengths (or listed); then packed Q [total_q, Hq, D], K and V
@@ -40,7 +44,7 @@ __all__ = ["PrefillCase", "DecodeCase", "VarlenCase", "PREFILL_CASES", "DECODE_C
            "VARLEN_CASES", "PagedPrefillCase", "PAGED_PREFILL_CASES", "make_paged_prefill",
            "make_prefill",
            "make_decode", "make_varlen", "varlen_flops",
-           "sample_rows"]
+           "sample_rows", "hadamard_signs", "Fp8Case", "FP8_CASES"]
 
 _DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16}
 
@@ -327,4 +331,29 @@ PAGED_PREFILL_CASES = {
         num_pages=16 * 512, nq=(512,) * 16,
         nk=(1024, 8192, 2048, 4096, 3000, 6000, 5120, 1536, 7000, 2500, 4500, 8000, 1800, 3500,
             6500, 5000)),
+}
+
+
+def hadamard_signs(D: int, seed: int) -> torch.Tensor:
+    """D random signs (+1.0 / -1.0, float32) for the Walsh-Hadamard rotation of
+    an FP8 forward's queries and keys: ``rand(D) < 0.5`` from a generator seeded
+    with ``seed`` gives -1."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    return torch.where(torch.rand(D, generator=g) < 0.5, -1.0, 1.0).to(torch.float32)
+
+
+@dataclass(frozen=True)
+class Fp8Case:
+    """An FP8 forward workload: the bf16 inputs of a prefill case, quantised to
+    E4M3 by the library, with the rotation's signs drawn from ``sign_seed``
+    (None: no rotation)."""
+    name: str
+    prefill: PrefillCase
+    sign_seed: int | None = None
+
+
+FP8_CASES = {
+    "fp8_gqa_b1_hq32_hkv8_n8192_d128_causal": Fp8Case(
+        "fp8_gqa_b1_hq32_hkv8_n8192_d128_causal",
+        PREFILL_CASES["gqa_b1_hq32_hkv8_n8192_d128_causal"], sign_seed=12),
 }
