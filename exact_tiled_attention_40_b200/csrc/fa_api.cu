@@ -63,9 +63,9 @@ EncodeTiledFn get_encode_fn() {
 }
 }  // namespace
 
-int encode_tensor_map_16bit(CUtensorMap* m, const void* base, bool bf16, int rank,
-                            const uint64_t* dims, const uint64_t* strides_bytes,
-                            const uint32_t* box) {
+namespace {
+int encode_tensor_map(CUtensorMap* m, CUtensorMapDataType type, const void* base, int rank,
+                      const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return set_error(FA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   cuuint64_t d[5], st[4];
@@ -76,13 +76,27 @@ int encode_tensor_map_16bit(CUtensorMap* m, const void* base, bool bf16, int ran
     es[i] = 1;
     if (i + 1 < rank) st[i] = strides_bytes[i];
   }
-  CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                   static_cast<cuuint32_t>(rank), const_cast<void*>(base), d, st, bx, es,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  CUresult r = enc(m, type, static_cast<cuuint32_t>(rank), const_cast<void*>(base), d, st, bx,
+                   es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return set_error(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", int(r));
   return FA_OK;
+}
+}  // namespace
+
+int encode_tensor_map_16bit(CUtensorMap* m, const void* base, bool bf16, int rank,
+                            const uint64_t* dims, const uint64_t* strides_bytes,
+                            const uint32_t* box) {
+  return encode_tensor_map(
+      m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base, rank,
+      dims, strides_bytes, box);
+}
+
+int encode_tensor_map_u8(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                         const uint64_t* strides_bytes, const uint32_t* box) {
+  return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, rank, dims, strides_bytes,
+                           box);
 }
 
 namespace {
@@ -216,10 +230,58 @@ int paged_common(const void* q, const void* kcache, const void* vcache,
                     max_pages_per_seq * 16, D, scale, causal, bf16, stream, dev);
 }
 
+int quantize_common(const void* x, void* codes, float* scales, int Z, int N, int D,
+                    int group_rows, const float* signs, cudaStream_t stream) {
+  if (Z < 0 || N < 0) return set_error(FA_ERR_INVALID_ARG, "negative size");
+  if (D != 64 && D != 128)
+    return set_error(FA_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", D);
+  if (group_rows != 0 && group_rows != 128)
+    return set_error(FA_ERR_UNSUPPORTED, "group_rows must be 128 or 0 (got %d)", group_rows);
+  if (Z == 0) return FA_OK;
+  if (Z > 65535) return set_error(FA_ERR_UNSUPPORTED, "Z (%d) above 65535", Z);
+  if (!scales || (N > 0 && (!x || !codes))) return set_error(FA_ERR_INVALID_ARG, "null pointer");
+  if (N > 0 && (!aligned16(x) || !aligned16(codes)))
+    return set_error(FA_ERR_INVALID_ARG, "x and codes must be 16-byte aligned");
+  if (static_cast<long long>(N) * D * Z > (1LL << 40))
+    return set_error(FA_ERR_INVALID_ARG, "tensor too large");
+  int dev, rc;
+  if ((rc = current_sm100(&dev)) != FA_OK) return rc;
+  return launch_quantize_e4m3(x, codes, scales, Z, N, D, group_rows, signs, stream, dev);
+}
+
+int fwd_fp8_common(const void* q8, const void* k8, const void* v8, const float* q_scale,
+                   const float* k_scale, const float* v_scale, void* o, float* lse, int B, int Hq,
+                   int Hkv, int Nq, int Nk, int D, float scale, int causal, cudaStream_t stream) {
+  int rc = validate_fwd(q8, k8, v8, o, B, Hq, Hkv, Nq, Nk, D, scale, causal);
+  if (rc != FA_OK) return rc;
+  if (D != 128)
+    return set_error(FA_ERR_UNSUPPORTED, "the FP8 forward supports D == 128 only (got %d)", D);
+  if (B == 0 || Hq == 0 || Nq == 0) return FA_OK;
+  if (!q_scale || (Nk > 0 && (!k_scale || !v_scale)))
+    return set_error(FA_ERR_INVALID_ARG, "null scale pointer");
+  int dev;
+  if ((rc = current_sm100(&dev)) != FA_OK) return rc;
+  return launch_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, Hq, Hkv, Nq, Nk, scale,
+                        causal, stream, dev);
+}
+
 }  // namespace
 }  // namespace fa
 
 extern "C" {
+
+int fa_quantize_e4m3(const void* x, void* codes, float* scales, int Z, int N, int D,
+                     int group_rows, const float* signs, fa_stream_t stream) {
+  return fa::quantize_common(x, codes, scales, Z, N, D, group_rows, signs,
+                             reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale,
+               const float* k_scale, const float* v_scale, void* o, float* lse, int B, int Hq,
+               int Hkv, int Nq, int Nk, int D, float scale, int causal, fa_stream_t stream) {
+  return fa::fwd_fp8_common(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, Hq, Hkv, Nq, Nk, D,
+                            scale, causal, reinterpret_cast<cudaStream_t>(stream));
+}
 
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
            int Hkv, int Nq, int Nk, int D, float scale, int causal, fa_stream_t stream) {

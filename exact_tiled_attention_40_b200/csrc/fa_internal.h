@@ -21,6 +21,10 @@ int encode_tensor_map_16bit(CUtensorMap* m, const void* base, bool bf16, int ran
                             const uint64_t* dims, const uint64_t* strides_bytes,
                             const uint32_t* box);
 
+// The same over one-byte elements (E4M3 codes).
+int encode_tensor_map_u8(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                         const uint64_t* strides_bytes, const uint32_t* box);
+
 // Wall-time limit of every bounded wait inside a kernel.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
@@ -49,6 +53,18 @@ int launch_decode(const void* q, const void* kcache, const void* vcache, const i
                   const int32_t* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int D,
                   int page_size, float scale, int max_pages_per_seq, int num_pages,
                   cudaStream_t stream, int device);
+
+// E4M3 quantisation of a bf16 tensor [Z, N, D] (validated arguments): codes
+// [Z, N, D], fp32 scales [Z, ceil(N / 128)] (group_rows 128) or [Z] (0), with
+// the optional Walsh-Hadamard rotation by `signs` [D].
+int launch_quantize_e4m3(const void* x, void* codes, float* scales, int Z, int N, int D,
+                         int group_rows, const float* signs, cudaStream_t stream, int device);
+
+// FP8 (E4M3) forward prefill launcher (validated arguments, D = 128).
+int launch_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale,
+                   const float* k_scale, const float* v_scale, void* o, float* lse, int B,
+                   int Hq, int Hkv, int Nq, int Nk, float scale, int causal, cudaStream_t stream,
+                   int device);
 
 // Release cached per-device resources owned by the decode path.
 void release_decode_resources();

@@ -35,6 +35,8 @@ _SIGS = {
                                 _I, _P]),
     "fa_fwd_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I,
                           _F, _I, _P]),
+    "fa_quantize_e4m3": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P]),
+    "fa_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _I, _I, _P]),
     "fa_decode_paged_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _I, _I,
                                      _P]),
@@ -176,6 +178,74 @@ def prefill_paged(q, kcache, vcache, block_table, cu_seqlens_q, seq_lens_k, max_
                  int(max_seqlen_q), block_table.shape[1], num_pages, total_q, D, page_size, scale,
                  causal)
     return o, lse
+
+
+def fa_quantize_e4m3(x, codes, scales, Z, N, D, group_rows, signs=None, stream=None):
+    """Raw call of the E4M3 quantiser's C entry point."""
+    s = _stream(x.device) if stream is None else ctypes.c_void_p(stream)
+    _check(lib().fa_quantize_e4m3(_ptr(x), _ptr(codes), _ptr(scales), Z, N, D, group_rows,
+                                  _ptr(signs), s), "fa_quantize_e4m3")
+
+
+def quantize_e4m3(x: torch.Tensor, group_rows: int = 128, signs: torch.Tensor | None = None):
+    """E4M3 codes (uint8, x's shape) and fp32 scales of a bf16 CUDA tensor x [..., N, D]:
+    scales [prod(...), ceil(N / 128)] for group_rows 128, [prod(...)] for 0.  With
+    signs [D] (+-1 fp32), rows are rotated by diag(signs) H / sqrt(D) first."""
+    if not x.is_cuda or x.dtype != torch.bfloat16:
+        raise FAError(1, "quantize_e4m3", "x must be a bf16 CUDA tensor")
+    if signs is not None and (not signs.is_cuda or signs.dtype != torch.float32):
+        raise FAError(1, "quantize_e4m3", "signs must be an fp32 CUDA tensor")
+    x = x.contiguous()
+    *lead, N, D = x.shape
+    Z = 1
+    for d in lead:
+        Z *= d
+    codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    shape = (Z, -(-N // 128)) if group_rows == 128 else (Z,)
+    scales = torch.empty(shape, dtype=torch.float32, device=x.device)
+    fa_quantize_e4m3(x, codes, scales, Z, N, D, group_rows,
+                     None if signs is None else signs.contiguous())
+    return codes, scales
+
+
+def fa_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, Hq, Hkv, Nq, Nk, D, scale,
+               causal, stream=None):
+    """Raw call of the FP8 forward's C entry point."""
+    s = _stream(q8.device) if stream is None else ctypes.c_void_p(stream)
+    _check(lib().fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale),
+                            _ptr(v_scale), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, D, float(scale),
+                            int(bool(causal)), s), "fa_fwd_fp8")
+
+
+def attention_fp8_quantised(q8, k8, v8, q_scale, k_scale, v_scale, scale=None, causal=False,
+                            return_lse=True):
+    """O (bf16) and LSE from E4M3 codes q8 [B,Hq,Nq,128], k8, v8 [B,Hkv,Nk,128] (uint8) with
+    the scales quantize_e4m3 writes (q, k in 128-row groups, v per slice)."""
+    for t in (q8, k8, v8, q_scale, k_scale, v_scale):
+        if not t.is_cuda:
+            raise FAError(1, "attention_fp8", "tensors must live on a CUDA device")
+    if q8.dtype != torch.uint8 or k8.dtype != torch.uint8 or v8.dtype != torch.uint8:
+        raise FAError(1, "attention_fp8", "codes must be uint8")
+    B, Hq, Nq, D = q8.shape
+    _, Hkv, Nk, _ = k8.shape
+    if scale is None:
+        scale = D ** -0.5
+    o = torch.empty((B, Hq, Nq, D), dtype=torch.bfloat16, device=q8.device)
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q8.device) if return_lse else None
+    fa_fwd_fp8(q8.contiguous(), k8.contiguous(), v8.contiguous(), q_scale.contiguous(),
+               k_scale.contiguous(), v_scale.contiguous(), o, lse, B, Hq, Hkv, Nq, Nk, D, scale,
+               causal)
+    return o, lse
+
+
+def attention_fp8(q, k, v, scale=None, causal=False, signs=None, return_lse=True):
+    """FP8 attention of bf16 q [B,Hq,Nq,128], k, v [B,Hkv,Nk,128]: q and k quantised in
+    128-row groups (rotated by the Walsh-Hadamard map with `signs` when given), v per
+    (sequence, head), then the E4M3 forward.  Returns (O bf16, LSE fp32)."""
+    q8, qs = quantize_e4m3(q, 128, signs)
+    k8, ks = quantize_e4m3(k, 128, signs)
+    v8, vs = quantize_e4m3(v, 0)
+    return attention_fp8_quantised(q8, k8, v8, qs, ks, vs, scale, causal, return_lse)
 
 
 def fa_decode_paged(q, kcache, vcache, block_table, seq_lens, o, B, Hq, Hkv, D, page_size, scale,

@@ -137,6 +137,54 @@ int fa_fwd_paged(const void* q, const void* kcache, const void* vcache,
                  float scale, int causal, fa_stream_t stream);
 
 /*
+ * E4M3 (FP8) quantisation of a bf16 tensor, the input preparation of
+ * fa_fwd_fp8.  unite.ai, "Flash Attention: Revolutionizing Transformer
+ * Efficiency", section "Flash Attention-3", names FP8 inputs with block
+ * quantisation and incoherent processing without defining them; this entry
+ * point takes the plainest reading:
+ *   x       [Z, N, D] bf16 (Z slices of N rows, e.g. Z = B * H)
+ *   codes   [Z, N, D] uint8 E4M3 codes (written): sign bit 7, exponent bits 3-6
+ *           (bias 7), mantissa bits 0-2, largest finite value 448
+ *   scales  fp32 (written), x ~= code * scale of the row's group:
+ *           group_rows == 128: [Z, ceil(N / 128)], one per 128-row group;
+ *           group_rows == 0:   [Z], one per slice.
+ *   signs   [D] fp32 of +1.0 / -1.0, or NULL.  When given, every row is first
+ *           multiplied by diag(signs) H / sqrt(D) (H the Walsh-Hadamard matrix,
+ *           H[i][j] = (-1)^popcount(i & j)): an orthogonal map, applied to Q and
+ *           K alike, that leaves Q K^T unchanged and spreads outliers.
+ * Per group: amax = max |x| (after the rotation), scale = amax / 448 and
+ * r = 448 / amax (both rounded to fp32; 1 when amax == 0), code = E4M3 of the
+ * fp32 product x * r, rounded to nearest even, finite values beyond 448
+ * saturating.  The rotation runs in fp32 as the fast Walsh-Hadamard transform
+ * (butterfly stages in increasing bit order) after one fp32 product per element
+ * by sign / sqrt(D).  Supported: D in {64, 128}, group_rows in {128, 0},
+ * Z <= 65535.  group_rows == 0 takes three kernel launches and a memset of
+ * `scales` on `stream`; no workspace is allocated.  Inputs must be finite.
+ */
+int fa_quantize_e4m3(const void* x, void* codes, float* scales, int Z, int N, int D,
+                     int group_rows, const float* signs, fa_stream_t stream);
+
+/*
+ * FP8 (E4M3) prefill: O = softmax(scale * Q K^T [+ causal]) V on quantised
+ * inputs (section "Flash Attention-3" of the unite.ai page above: FP8 with
+ * block quantisation).
+ *   q8  [B, Hq,  Nq, 128] uint8 E4M3 codes, q_scale [B * Hq,  ceil(Nq / 128)] fp32
+ *   k8  [B, Hkv, Nk, 128] uint8 E4M3 codes, k_scale [B * Hkv, ceil(Nk / 128)] fp32
+ *   v8  [B, Hkv, Nk, 128] uint8 E4M3 codes, v_scale [B * Hkv] fp32
+ *   o   [B, Hq, Nq, 128] bf16 (written), lse [B, Hq, Nq] fp32 (written; may be NULL)
+ * i.e. exactly what fa_quantize_e4m3 writes for group_rows 128 (q, k) and 0 (v);
+ * the inputs represent q8 * q_scale of the row's 128-row group, and so on.
+ * Scales must be positive and finite (other values give unspecified numbers,
+ * never an out-of-range access).  Causal masking, GQA and the argument rules
+ * are those of fa_fwd; D == 128 only.  Q K^T and P V run on the tensor cores
+ * in E4M3 with fp32 accumulation; P is rounded to E4M3 before P V (at most
+ * 2^-4 relative error per normal entry), the row sums are kept in fp32.
+ */
+int fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale,
+               const float* k_scale, const float* v_scale, void* o, float* lse, int B, int Hq,
+               int Hkv, int Nq, int Nk, int D, float scale, int causal, fa_stream_t stream);
+
+/*
  * Decode over a paged KV cache: one new query token per sequence attends over
  * all of that sequence's cached keys and values (no mask beyond its length).
  *   q           [B, Hq, D] bf16

@@ -137,3 +137,65 @@ def test_paged_prefill_rejects_bad_arguments_on_the_host(lib, kw, code):
 def test_paged_prefill_empty_batch_is_a_noop(lib):
     assert paged(lib, B=0) == 0
     assert paged(lib, tq=0) == 0
+
+
+def quant(lib, x=FAKE, codes=FAKE, scales=FAKE, Z=4, N=300, D=128, group=128, signs=None):
+    return lib.fa_quantize_e4m3(x, codes, scales, Z, N, D, group, signs, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Z=-1), "FA_ERR_INVALID_ARG"),
+    (dict(N=-5), "FA_ERR_INVALID_ARG"),
+    (dict(D=96), "FA_ERR_UNSUPPORTED"),
+    (dict(group=64), "FA_ERR_UNSUPPORTED"),
+    (dict(Z=70000), "FA_ERR_UNSUPPORTED"),
+    (dict(x=None), "FA_ERR_INVALID_ARG"),
+    (dict(codes=None), "FA_ERR_INVALID_ARG"),
+    (dict(scales=None), "FA_ERR_INVALID_ARG"),
+    (dict(x=FAKE + 8), "FA_ERR_INVALID_ARG"),
+    (dict(codes=FAKE + 1), "FA_ERR_INVALID_ARG"),
+])
+def test_quantize_rejects_bad_arguments_on_the_host(lib, kw, code):
+    assert quant(lib, **kw) == E[code]
+    assert lib.fa_last_error_string()
+
+
+def test_quantize_empty_slices_need_no_data_pointers(lib):
+    assert quant(lib, Z=0) == 0
+    # N == 0 still writes scales (1 per slice for group 0), so it reaches the device
+    assert quant(lib, N=0, x=None, codes=None) in (0, E["FA_ERR_NO_DEVICE"])
+
+
+def fp8(lib, B=1, Hq=2, Hkv=1, Nq=8, Nk=8, D=128, scale=0.1, causal=0, q=FAKE, k=FAKE,
+        v=FAKE, qs=FAKE, ks=FAKE, vs=FAKE, o=FAKE):
+    return lib.fa_fwd_fp8(q, k, v, qs, ks, vs, o, None, B, Hq, Hkv, Nq, Nk, D, scale, causal,
+                          None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=-1), "FA_ERR_INVALID_ARG"),
+    (dict(D=64), "FA_ERR_UNSUPPORTED"),
+    (dict(D=96), "FA_ERR_UNSUPPORTED"),
+    (dict(Hq=3, Hkv=2), "FA_ERR_INVALID_ARG"),
+    (dict(causal=1, Nq=9, Nk=8), "FA_ERR_INVALID_ARG"),
+    (dict(scale=0.0), "FA_ERR_INVALID_ARG"),
+    (dict(q=0), "FA_ERR_INVALID_ARG"),
+    (dict(v=FAKE + 4), "FA_ERR_INVALID_ARG"),
+    (dict(qs=None), "FA_ERR_INVALID_ARG"),
+    (dict(ks=None), "FA_ERR_INVALID_ARG"),
+    (dict(vs=None), "FA_ERR_INVALID_ARG"),
+])
+def test_fp8_forward_rejects_bad_arguments_on_the_host(lib, kw, code):
+    assert fp8(lib, **kw) == E[code]
+    assert lib.fa_last_error_string()
+
+
+def test_fp8_forward_empty_problem_is_a_noop(lib):
+    assert fp8(lib, B=0) == 0
+    assert fp8(lib, Nq=0) == 0
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_fp8_calls_without_a_device_fail_loudly(lib):
+    assert fp8(lib) == E["FA_ERR_NO_DEVICE"]
+    assert quant(lib) == E["FA_ERR_NO_DEVICE"]
