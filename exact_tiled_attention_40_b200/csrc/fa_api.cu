@@ -265,10 +265,32 @@ int fwd_fp8_common(const void* q8, const void* k8, const void* v8, const float* 
                         causal, stream, dev);
 }
 
+int merge_common(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+                 void* o_out, long long rows, int D, int first, cudaStream_t stream) {
+  if (rows < 0) return set_error(FA_ERR_INVALID_ARG, "negative size");
+  if (D != 64 && D != 128)
+    return set_error(FA_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", D);
+  if (rows == 0) return FA_OK;
+  if (!o_acc || !lse_acc || !o_part || !lse_part)
+    return set_error(FA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(o_acc) || !aligned16(o_part) || (o_out && !aligned16(o_out)))
+    return set_error(FA_ERR_INVALID_ARG, "o_acc, o_part and o_out must be 16-byte aligned");
+  int dev, rc;
+  if ((rc = current_sm100(&dev)) != FA_OK) return rc;
+  return launch_merge_partials(o_acc, lse_acc, o_part, lse_part, o_out, rows, D, first ? 1 : 0,
+                               stream, dev);
+}
+
 }  // namespace
 }  // namespace fa
 
 extern "C" {
+
+int fa_merge_partials(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+                      void* o_out, long long rows, int D, int first, fa_stream_t stream) {
+  return fa::merge_common(o_acc, lse_acc, o_part, lse_part, o_out, rows, D, first,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
 
 int fa_quantize_e4m3(const void* x, void* codes, float* scales, int Z, int N, int D,
                      int group_rows, const float* signs, fa_stream_t stream) {

@@ -66,6 +66,13 @@ int launch_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* 
                    int Hq, int Hkv, int Nq, int Nk, float scale, int causal, cudaStream_t stream,
                    int device);
 
+// Merge of a partial attention result (o_part bf16 [rows, D], lse_part) into an
+// fp32 accumulator (o_acc [rows, D], lse_acc; overwritten when `first`), with
+// an optional bf16 copy of the merged rows (validated arguments).
+int launch_merge_partials(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+                          void* o_out, long long rows, int D, int first, cudaStream_t stream,
+                          int device);
+
 // Release cached per-device resources owned by the decode path.
 void release_decode_resources();
 

@@ -37,6 +37,7 @@ _SIGS = {
                           _F, _I, _P]),
     "fa_quantize_e4m3": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P]),
     "fa_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_merge_partials": (_I, [_P, _P, _P, _P, _P, ctypes.c_longlong, _I, _I, _P]),
     "fa_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _I, _I, _P]),
     "fa_decode_paged_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _I, _I,
                                      _P]),
@@ -246,6 +247,30 @@ def attention_fp8(q, k, v, scale=None, causal=False, signs=None, return_lse=True
     k8, ks = quantize_e4m3(k, 128, signs)
     v8, vs = quantize_e4m3(v, 0)
     return attention_fp8_quantised(q8, k8, v8, qs, ks, vs, scale, causal, return_lse)
+
+
+def merge_partials(o_acc, lse_acc, o_part, lse_part, first=False, o_out=None, stream=None):
+    """Fold a partial result (o_part bf16 [..., D], lse_part fp32 [...]) into the fp32
+    accumulator (o_acc [..., D], lse_acc [...]) by their LSE, in place; with `o_out`
+    (bf16, o_part's shape) the merged rows are also written there."""
+    for t in (o_acc, lse_acc, o_part, lse_part):
+        if not t.is_cuda or not t.is_contiguous():
+            raise FAError(1, "merge_partials", "tensors must be contiguous CUDA tensors")
+    if o_acc.dtype != torch.float32 or lse_acc.dtype != torch.float32 or \
+            lse_part.dtype != torch.float32 or o_part.dtype != torch.bfloat16:
+        raise FAError(1, "merge_partials", "o_acc, lse fp32 and o_part bf16 expected")
+    if o_acc.shape != o_part.shape or lse_acc.shape != lse_part.shape or \
+            o_part.shape[:-1] != lse_part.shape:
+        raise FAError(1, "merge_partials", "shape mismatch")
+    if o_out is not None and (o_out.shape != o_part.shape or o_out.dtype != torch.bfloat16
+                              or not o_out.is_contiguous()):
+        raise FAError(1, "merge_partials", "o_out must be a contiguous bf16 tensor like o_part")
+    D = o_part.shape[-1]
+    rows = lse_part.numel()
+    s = _stream(o_part.device) if stream is None else ctypes.c_void_p(stream)
+    _check(lib().fa_merge_partials(_ptr(o_acc), _ptr(lse_acc), _ptr(o_part), _ptr(lse_part),
+                                   _ptr(o_out), rows, D, int(bool(first)), s),
+           "fa_merge_partials")
 
 
 def fa_decode_paged(q, kcache, vcache, block_table, seq_lens, o, B, Hq, Hkv, D, page_size, scale,

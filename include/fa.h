@@ -185,6 +185,25 @@ int fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_sc
                int Hkv, int Nq, int Nk, int D, float scale, int causal, fa_stream_t stream);
 
 /*
+ * Merge of partial attention results over disjoint key sets (the combine step
+ * of the split-KV decode, exposed for sequence-sharded prefill: each rank's
+ * queries meet the K/V chunks of every rank and fold each chunk's result in).
+ * unite.ai page above, section "The Mathematics of Flash Attention": with
+ * normalised partial outputs and their log-sum-exps,
+ *     lse = log(e^lse_acc + e^lse_part),
+ *     O   = e^(lse_acc - lse) O_acc + e^(lse_part - lse) O_part.
+ *   o_acc    [rows, D] fp32, read (unless `first`) and written
+ *   lse_acc  [rows] fp32, read (unless `first`) and written; -inf = no key yet
+ *   o_part   [rows, D] bf16 (e.g. fa_fwd's output over one key chunk)
+ *   lse_part [rows] fp32 (fa_fwd's LSE over that chunk; -inf = no key)
+ *   o_out    [rows, D] bf16, written with the merged rows when not NULL
+ *   first    nonzero: the accumulator is set to the part (o_acc, lse_acc not read)
+ * Rows where both LSEs are -inf get O = 0, LSE = -inf.  D in {64, 128}.
+ */
+int fa_merge_partials(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+                      void* o_out, long long rows, int D, int first, fa_stream_t stream);
+
+/*
  * Decode over a paged KV cache: one new query token per sequence attends over
  * all of that sequence's cached keys and values (no mask beyond its length).
  *   q           [B, Hq, D] bf16

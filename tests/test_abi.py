@@ -199,3 +199,23 @@ def test_fp8_forward_empty_problem_is_a_noop(lib):
 def test_fp8_calls_without_a_device_fail_loudly(lib):
     assert fp8(lib) == E["FA_ERR_NO_DEVICE"]
     assert quant(lib) == E["FA_ERR_NO_DEVICE"]
+
+
+def merge(lib, oa=FAKE, la=FAKE, op=FAKE, lp=FAKE, out=None, rows=10, D=128, first=0):
+    return lib.fa_merge_partials(oa, la, op, lp, out, rows, D, first, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(rows=-1), "FA_ERR_INVALID_ARG"),
+    (dict(D=96), "FA_ERR_UNSUPPORTED"),
+    (dict(oa=None), "FA_ERR_INVALID_ARG"),
+    (dict(lp=None), "FA_ERR_INVALID_ARG"),
+    (dict(op=FAKE + 2), "FA_ERR_INVALID_ARG"),
+    (dict(out=FAKE + 4), "FA_ERR_INVALID_ARG"),
+])
+def test_merge_rejects_bad_arguments_on_the_host(lib, kw, code):
+    assert merge(lib, **kw) == E[code]
+
+
+def test_merge_of_no_rows_is_a_noop(lib):
+    assert merge(lib, rows=0, oa=None, op=None) == 0
