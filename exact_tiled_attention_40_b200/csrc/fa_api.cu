@@ -281,10 +281,47 @@ int merge_common(float* o_acc, float* lse_acc, const void* o_part, const float* 
                                stream, dev);
 }
 
+int bwd_common(const void* q, const void* k, const void* v, const void* o, const float* lse,
+               const void* dout, void* dq, void* dk, void* dv, float* delta, int B, int Hq,
+               int Hkv, int Nq, int Nk, int D, float scale, int causal, cudaStream_t stream) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || Nq < 0 || Nk < 0)
+    return set_error(FA_ERR_INVALID_ARG, "negative size");
+  if (!(std::isfinite(scale) && scale > 0.f))
+    return set_error(FA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (D != 64 && D != 128)
+    return set_error(FA_ERR_UNSUPPORTED, "head dimension %d is not supported (64 or 128)", D);
+  if (B == 0 || Hq == 0 || (Nq == 0 && Nk == 0)) return FA_OK;
+  if (Hkv <= 0 || Hq % Hkv != 0)
+    return set_error(FA_ERR_INVALID_ARG, "Hq (%d) must be a positive multiple of Hkv (%d)", Hq,
+                     Hkv);
+  if (causal && Nq > Nk)
+    return set_error(FA_ERR_INVALID_ARG, "causal attention needs Nq <= Nk (got %d > %d)", Nq, Nk);
+  const bool has_q = Nq > 0, has_k = Nk > 0;
+  if ((has_q && (!q || !o || !lse || !dout || !dq || !delta)) ||
+      (has_k && (!k || !v || !dk || !dv)))
+    return set_error(FA_ERR_INVALID_ARG, "null pointer");
+  if ((has_q && (!aligned16(q) || !aligned16(o) || !aligned16(dout) || !aligned16(dq))) ||
+      (has_k && (!aligned16(k) || !aligned16(v) || !aligned16(dk) || !aligned16(dv))))
+    return set_error(FA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (static_cast<long long>(B) * Hq > 0x7fffffffLL)
+    return set_error(FA_ERR_UNSUPPORTED, "B * H too large");
+  int dev, rc;
+  if ((rc = current_sm100(&dev)) != FA_OK) return rc;
+  return launch_bwd(q, k, v, o, lse, dout, dq, dk, dv, delta, B, Hq, Hkv, Nq, Nk, D, scale,
+                    causal, stream, dev);
+}
+
 }  // namespace
 }  // namespace fa
 
 extern "C" {
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dout, void* dq, void* dk, void* dv, float* delta, int B, int Hq, int Hkv,
+           int Nq, int Nk, int D, float scale, int causal, fa_stream_t stream) {
+  return fa::bwd_common(q, k, v, o, lse, dout, dq, dk, dv, delta, B, Hq, Hkv, Nq, Nk, D, scale,
+                        causal, reinterpret_cast<cudaStream_t>(stream));
+}
 
 int fa_merge_partials(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
                       void* o_out, long long rows, int D, int first, fa_stream_t stream) {

@@ -1,0 +1,702 @@
+// Exact attention backward for sm_100a, with recomputation.
+//
+// unite.ai, "Flash Attention: Revolutionizing Transformer Efficiency", names
+// recomputation in the backward pass (the N x N probabilities are not stored;
+// the forward keeps only O and the per-row log-sum-exp, from which P is rebuilt
+// tile by tile).  With P = exp(scale Q K^T - LSE) and the row sums
+// delta_i = sum_d dO_id O_id:
+//     dV = P^T dO,  dP = dO V^T,  dS = P * (dP - delta),
+//     dQ = scale dS K,  dK = scale dS^T Q,
+// GQA: the query heads of one KV head add into its dK, dV.
+//
+// Three kernels, no atomics and no workspace beyond delta:
+//   fa_bwd_delta_kernel  delta = rowsum(dO * O) (a warp per row, HBM-bound).
+//   fa_bwd_dkdv_kernel   one CTA per (sequence, KV head, 128-key tile j): K_j, V_j
+//                        stay in shared memory; the Q_i, dO_i tiles of every query
+//                        head of the group stream through a two-slot ring.  Per
+//                        tile pair the MMA warp computes S^T = K_j Q_i^T and
+//                        dP^T = V_j dO_i^T into TMEM; the 128 softmax threads
+//                        (thread r = key r = TMEM lane r) rebuild P^T and dS^T and
+//                        write them back over the first halves of those TMEM
+//                        columns as bf16 pairs; the MMA warp then accumulates
+//                        dV += P^T dO_i and dK += dS^T Q_i (A operand from TMEM).
+//   fa_bwd_dq_kernel     one CTA per (sequence, query head, 128-row tile i): Q_i,
+//                        dO_i stay; K_j, V_j stream.  S = Q_i K_j^T and
+//                        dP = dO_i V_j^T into TMEM, dS (per row: its own LSE and
+//                        delta) back as bf16, dQ += dS K_j.
+// Each recomputes S and dP, seven tile products per pair instead of five, in
+// exchange for no atomics and a TMEM budget that fits (dK/dV kernel: S^T, dP^T,
+// dV, dK = 4 x 128 columns at D = 128; dQ kernel: S, dP, dQ).
+// Warps: 0-3 softmax (one TMEM lane quarter each), 4 TMA producer, 5 MMA issuer
+// (an elected lane issues).  Every wait is bounded (mbar_wait).
+#include <algorithm>
+#include <cfloat>
+#include <cstdio>
+#include <mutex>
+
+#include "fa_internal.h"
+#include "ptx_sm100.cuh"
+#include "../../include/fa.h"
+
+namespace fa {
+namespace {
+
+constexpr int kBM = 128;                  // rows of every tile (TMEM lanes)
+constexpr int kThreads = 192;             // 4 softmax warps, producer, MMA
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct BwdLayout {
+  static constexpr int kChunks = D / 64;                // 128-byte swizzle atoms along D
+  static constexpr int kChunkBytes = kBM * 128;
+  static constexpr int kTileBytes = kBM * D * 2;
+  // two stationary tiles, then a two-slot ring of tile pairs
+  static constexpr int kFixOff = 0;
+  static constexpr int kRingOff = 2 * kTileBytes;
+  static constexpr int kBarOff = kRingOff + 4 * kTileBytes;
+  static constexpr int kNumBars = 1 + 2 + 2 + 1 + 1 + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+struct BwdParams {
+  const uint16_t* o;
+  const uint16_t* dout;
+  const float* lse;      // [B * Hq, Nq], natural log
+  float* delta;          // [B * Hq, Nq]
+  uint16_t* dq;
+  uint16_t* dk;
+  uint16_t* dv;
+  int B, Hq, Hkv, Nq, Nk;
+  int causal;
+  float scale;
+  float scale_log2;      // scale * log2(e)
+  int* err;
+  uint64_t timeout_ns;
+};
+
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// delta[row] = sum_d dO[row, d] * O[row, d]; a warp per row.
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_delta_kernel(const uint16_t* __restrict__ o,
+                                                           const uint16_t* __restrict__ dout,
+                                                           float* __restrict__ delta,
+                                                           long long rows) {
+  constexpr int E = D / 32;
+  const int lane = threadIdx.x & 31;
+  const long long warps = static_cast<long long>(gridDim.x) * 8;
+  for (long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5); row < rows;
+       row += warps) {
+    const size_t base = static_cast<size_t>(row) * D + lane * E;
+    float acc = 0.f;
+    if constexpr (E == 4) {
+      const uint2 a = __ldg(reinterpret_cast<const uint2*>(o + base));
+      const uint2 b = __ldg(reinterpret_cast<const uint2*>(dout + base));
+      acc = bf_lo(a.x) * bf_lo(b.x) + bf_hi(a.x) * bf_hi(b.x) + bf_lo(a.y) * bf_lo(b.y) +
+            bf_hi(a.y) * bf_hi(b.y);
+    } else {
+      const uint32_t a = __ldg(reinterpret_cast<const uint32_t*>(o + base));
+      const uint32_t b = __ldg(reinterpret_cast<const uint32_t*>(dout + base));
+      acc = bf_lo(a) * bf_lo(b) + bf_hi(a) * bf_hi(b);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) delta[row] = acc;
+  }
+}
+
+// K-major descriptor step kk (16 elements of D) inside a [128, D] tile.
+template <int D>
+__device__ __forceinline__ uint64_t kmajor_step(int kk) {
+  return static_cast<uint64_t>(((kk >> 2) * BwdLayout<D>::kChunkBytes + (kk & 3) * 32) >> 4);
+}
+
+// 128 x 128 product of two K-major [128, D] tiles (rows of A against rows of B)
+// into TMEM columns d .. d + 127.
+template <int D>
+__device__ __forceinline__ void mma_rows_x_rows(uint32_t d, uint64_t a, uint64_t b) {
+  constexpr uint32_t idesc = idesc_f16(kBM, kBM, true, false);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk)
+    mma_ss(d, a + kmajor_step<D>(kk), b + kmajor_step<D>(kk), idesc, kk > 0 ? 1u : 0u);
+}
+
+// D-column accumulation: TMEM[d .. d + D) (+)= A (bf16 pairs in TMEM columns
+// a .. a + 63, 128 K values) x B ([128, D] tile read MN-major).
+template <int D>
+__device__ __forceinline__ void mma_tmem_x_tile(uint32_t d, uint32_t a, uint64_t b_mn,
+                                                bool accumulate) {
+  constexpr uint32_t idesc = idesc_f16(kBM, D, true, true);
+#pragma unroll
+  for (int kk = 0; kk < kBM / 16; ++kk)
+    mma_ts(d, a + kk * 8, b_mn + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc,
+           (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// Store a row of D fp32 TMEM values (columns t0 ..), times `mul`, as bf16.
+template <int D>
+__device__ __forceinline__ void store_row_bf16(uint32_t t0, float mul, uint16_t* dst, bool valid) {
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t v[32];
+    tmem_ld32(t0 + 32 * c, v);
+    tmem_wait_ld();
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+    if (valid) {
+      uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        d4[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+    }
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void store_zero_row(uint16_t* dst) {
+  const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(dst)[c] = z;
+}
+
+// First query tile that sees key tile j (causal, bottom-right aligned).
+__device__ __forceinline__ int first_q_tile(int j, int Nq, int Nk, int causal) {
+  if (!causal) return 0;
+  const int t = j * kBM - (Nk - Nq);   // the first query row that sees key j * 128
+  return t <= 0 ? 0 : t / kBM;
+}
+
+// ---------------------------------------------------------------- dK, dV
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV,
+                       const __grid_constant__ CUtensorMap tmdO, const BwdParams p) {
+  using L = BwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+
+  // work: key tile j of (b, hkv)
+  const int n_kt = (p.Nk + kBM - 1) / kBM;
+  const int j = blockIdx.x % n_kt;
+  const int bh_kv = blockIdx.x / n_kt;
+  const int b = bh_kv / p.Hkv;
+  const int hkv = bh_kv - b * p.Hkv;
+  const int G = p.Hq / p.Hkv;
+  const int n_qt = (p.Nq + kBM - 1) / kBM;
+  const int i0 = first_q_tile(j, p.Nq, p.Nk, p.causal);
+  const int per_head = i0 < n_qt ? n_qt - i0 : 0;
+  const int n_items = per_head * G;     // (query head g, query tile i0 + t)
+  const int off = p.Nk - p.Nq;
+
+  auto bar = [&](int i) -> uint32_t { return sbase + L::kBarOff + 8 * i; };
+  const uint32_t kv_full = bar(0);
+  auto q_full = [&](int s) { return bar(1 + s); };
+  auto q_empty = [&](int s) { return bar(3 + s); };
+  const uint32_t s_full = bar(5);
+  const uint32_t p_full = bar(6);
+  const uint32_t acc_done = bar(7);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  const uint32_t k_smem = sbase + L::kFixOff;
+  const uint32_t v_smem = sbase + L::kFixOff + L::kTileBytes;
+  auto q_smem = [&](int s) { return sbase + L::kRingOff + (2 * s) * L::kTileBytes; };
+  auto do_smem = [&](int s) { return sbase + L::kRingOff + (2 * s + 1) * L::kTileBytes; };
+
+  if (tid == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(q_full(s), 1);
+      mbar_init(q_empty(s), 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, kBM);
+    mbar_init(acc_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // TMEM: [0,128) S^T then P^T (bf16 pairs in [0,64)); [128,256) dP^T then dS^T;
+  // [256,256+D) dV; [256+D,256+2D) dK
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && n_items > 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmdO);
+      mbar_arrive_expect_tx(kv_full, 2 * L::kTileBytes);
+      const int z_kv = b * p.Hkv + hkv;
+      for (int ch = 0; ch < L::kChunks; ++ch) {
+        tma_load_3d(k_smem + ch * L::kChunkBytes, &tmK, kv_full, ch * 64, j * kBM, z_kv);
+        tma_load_3d(v_smem + ch * L::kChunkBytes, &tmV, kv_full, ch * 64, j * kBM, z_kv);
+      }
+      int it = 0;
+      for (; it < n_items; ++it) {
+        const int s = it & 1;
+        if (!mbar_wait(q_empty(s), ((it >> 1) & 1) ^ 1, abort_flag, p.err, p.timeout_ns)) break;
+        const int g = it / per_head;
+        const int i = i0 + (it - g * per_head);
+        const int z = b * p.Hq + hkv * G + g;
+        mbar_arrive_expect_tx(q_full(s), 2 * L::kTileBytes);
+        for (int ch = 0; ch < L::kChunks; ++ch) {
+          tma_load_3d(q_smem(s) + ch * L::kChunkBytes, &tmQ, q_full(s), ch * 64, i * kBM, z);
+          tma_load_3d(do_smem(s) + ch * L::kChunkBytes, &tmdO, q_full(s), ch * 64, i * kBM, z);
+        }
+      }
+      // every issued copy lands before the CTA may exit
+      volatile int no_abort = 0;
+      mbar_wait(kv_full, 0, &no_abort, p.err, p.timeout_ns);
+      for (int s = 0; s < 2 && s < it; ++s) {
+        const int last = s + ((it - 1 - s) / 2) * 2;
+        mbar_wait(q_full(s), (last >> 1) & 1, &no_abort, p.err, p.timeout_ns);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    const bool leader = elect_one();
+    auto wait = [&](uint32_t br, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(br, parity, abort_flag, p.err, p.timeout_ns));
+    };
+    const uint64_t k_desc = smem_desc_sw128(k_smem, 16, 1024);
+    const uint64_t v_desc = smem_desc_sw128(v_smem, 16, 1024);
+    bool ok = n_items == 0 || wait(kv_full, 0);
+    for (int it = 0; ok && it < n_items; ++it) {
+      const int s = it & 1;
+      ok = wait(q_full(s), (it >> 1) & 1);
+      if (!ok) break;
+      tc_fence_after();
+      const uint64_t q_kdesc = smem_desc_sw128(q_smem(s), 16, 1024);
+      const uint64_t do_kdesc = smem_desc_sw128(do_smem(s), 16, 1024);
+      if (leader) {
+        mma_rows_x_rows<D>(tmem + 0, k_desc, q_kdesc);       // S^T = K_j Q_i^T
+        mma_rows_x_rows<D>(tmem + 128, v_desc, do_kdesc);    // dP^T = V_j dO_i^T
+        tc_commit(s_full);
+      }
+      ok = wait(p_full, it & 1);
+      if (!ok) break;
+      tc_fence_after();
+      const uint64_t q_mn = smem_desc_sw128(q_smem(s), L::kChunkBytes, 1024);
+      const uint64_t do_mn = smem_desc_sw128(do_smem(s), L::kChunkBytes, 1024);
+      if (leader) {
+        mma_tmem_x_tile<D>(tmem + 256, tmem + 0, do_mn, it > 0);        // dV += P^T dO_i
+        mma_tmem_x_tile<D>(tmem + 256 + D, tmem + 128, q_mn, it > 0);   // dK += dS^T Q_i
+        tc_commit(q_empty(s));
+      }
+    }
+    if (leader) tc_commit(acc_done);
+    volatile int no_abort = 0;
+    mbar_wait(acc_done, 0, &no_abort, p.err, p.timeout_ns);
+  } else {
+    // ------------------------------------------------------------ softmax warpgroup
+    const int r = tid;                                  // key row within the tile
+    const int kr = j * kBM + r;                         // key index
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tS = tmem + lane_base;
+    const uint32_t tP = tmem + lane_base + 128;
+    bool ok = true;
+    for (int it = 0; ok && it < n_items; ++it) {
+      const int g = it / per_head;
+      const int i = i0 + (it - g * per_head);
+      const size_t qrow0 = static_cast<size_t>(b * p.Hq + hkv * G + g) * p.Nq;
+      const bool got = mbar_wait(s_full, it & 1, abort_flag, p.err, p.timeout_ns);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // queries q0 + e of this chunk are visible to key kr when kr <= q + off
+      const bool band = p.causal && (j * kBM + kBM - 1 > i * kBM + off);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sv[32], dv[32];
+        tmem_ld32(tS + 32 * c, sv);
+        tmem_ld32(tP + 32 * c, dv);
+        tmem_wait_ld();
+        const int q0 = i * kBM + 32 * c;
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float pe[2], de[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int q = q0 + e + u;
+            float lse = INFINITY, dl = 0.f;
+            if (q < p.Nq) {
+              lse = __ldg(p.lse + qrow0 + q);
+              dl = __ldg(p.delta + qrow0 + q);
+            }
+            float pv = ex2(fmaf(__uint_as_float(sv[e + u]), p.scale_log2, -lse * kLog2e));
+            if (band && kr > q + off) pv = 0.f;
+            pe[u] = pv;
+            de[u] = pv * (__uint_as_float(dv[e + u]) - dl);
+          }
+          pk[e >> 1] = pack_bf16x2(pe[0], pe[1]);
+          dk[e >> 1] = pack_bf16x2(de[0], de[1]);
+        }
+        // the packed pairs go over columns already read (16 c .. 16 c + 15)
+        tmem_st16(tS + 16 * c, pk);
+        tmem_st16(tP + 16 * c, dk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    const bool fin = ok && (n_items == 0 ||
+                            mbar_wait(acc_done, 0, abort_flag, p.err, p.timeout_ns));
+    if (__all_sync(0xffffffffu, fin)) {
+      tc_fence_after();
+      const size_t orow = (static_cast<size_t>(b * p.Hkv + hkv) * p.Nk + kr) * D;
+      const bool valid = kr < p.Nk;
+      if (n_items == 0) {
+        if (valid) {
+          store_zero_row<D>(p.dv + orow);
+          store_zero_row<D>(p.dk + orow);
+        }
+      } else {
+        store_row_bf16<D>(tmem + lane_base + 256, 1.f, p.dv + orow, valid);
+        store_row_bf16<D>(tmem + lane_base + 256 + D, p.scale, p.dk + orow, valid);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- dQ
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ,
+                     const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV,
+                     const __grid_constant__ CUtensorMap tmdO, const BwdParams p) {
+  using L = BwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+
+  const int n_qt = (p.Nq + kBM - 1) / kBM;
+  const int i = blockIdx.x % n_qt;
+  const int bh = blockIdx.x / n_qt;                  // b * Hq + h
+  const int b = bh / p.Hq;
+  const int h = bh - b * p.Hq;
+  const int hkv = h / (p.Hq / p.Hkv);
+  const int off = p.Nk - p.Nq;
+  int n_kt = (p.Nk + kBM - 1) / kBM;
+  if (p.causal) {
+    const int last_row = min(i * kBM + kBM - 1, p.Nq - 1);
+    n_kt = min(n_kt, (last_row + off) / kBM + 1);
+  }
+
+  auto bar = [&](int x) -> uint32_t { return sbase + L::kBarOff + 8 * x; };
+  const uint32_t q_full = bar(0);
+  auto kv_full = [&](int s) { return bar(1 + s); };
+  auto kv_empty = [&](int s) { return bar(3 + s); };
+  const uint32_t s_full = bar(5);
+  const uint32_t ds_full = bar(6);
+  const uint32_t acc_done = bar(7);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  const uint32_t q_smem = sbase + L::kFixOff;
+  const uint32_t do_smem = sbase + L::kFixOff + L::kTileBytes;
+  auto k_smem = [&](int s) { return sbase + L::kRingOff + (2 * s) * L::kTileBytes; };
+  auto v_smem = [&](int s) { return sbase + L::kRingOff + (2 * s + 1) * L::kTileBytes; };
+
+  if (tid == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(kv_full(s), 1);
+      mbar_init(kv_empty(s), 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(ds_full, kBM);
+    mbar_init(acc_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // TMEM: [0,128) S then dS (bf16 pairs in [0,64)); [128,256) dP; [256,256+D) dQ
+
+  if (warp == 4) {
+    if (lane == 0 && n_kt > 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmdO);
+      mbar_arrive_expect_tx(q_full, 2 * L::kTileBytes);
+      for (int ch = 0; ch < L::kChunks; ++ch) {
+        tma_load_3d(q_smem + ch * L::kChunkBytes, &tmQ, q_full, ch * 64, i * kBM, bh);
+        tma_load_3d(do_smem + ch * L::kChunkBytes, &tmdO, q_full, ch * 64, i * kBM, bh);
+      }
+      const int z_kv = b * p.Hkv + hkv;
+      int jt = 0;
+      for (; jt < n_kt; ++jt) {
+        const int s = jt & 1;
+        if (!mbar_wait(kv_empty(s), ((jt >> 1) & 1) ^ 1, abort_flag, p.err, p.timeout_ns)) break;
+        mbar_arrive_expect_tx(kv_full(s), 2 * L::kTileBytes);
+        for (int ch = 0; ch < L::kChunks; ++ch) {
+          tma_load_3d(k_smem(s) + ch * L::kChunkBytes, &tmK, kv_full(s), ch * 64, jt * kBM, z_kv);
+          tma_load_3d(v_smem(s) + ch * L::kChunkBytes, &tmV, kv_full(s), ch * 64, jt * kBM, z_kv);
+        }
+      }
+      volatile int no_abort = 0;
+      mbar_wait(q_full, 0, &no_abort, p.err, p.timeout_ns);
+      for (int s = 0; s < 2 && s < jt; ++s) {
+        const int last = s + ((jt - 1 - s) / 2) * 2;
+        mbar_wait(kv_full(s), (last >> 1) & 1, &no_abort, p.err, p.timeout_ns);
+      }
+    }
+  } else if (warp == 5) {
+    const bool leader = elect_one();
+    auto wait = [&](uint32_t br, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(br, parity, abort_flag, p.err, p.timeout_ns));
+    };
+    const uint64_t q_desc = smem_desc_sw128(q_smem, 16, 1024);
+    const uint64_t do_desc = smem_desc_sw128(do_smem, 16, 1024);
+    bool ok = n_kt == 0 || wait(q_full, 0);
+    for (int jt = 0; ok && jt < n_kt; ++jt) {
+      const int s = jt & 1;
+      ok = wait(kv_full(s), (jt >> 1) & 1);
+      if (!ok) break;
+      tc_fence_after();
+      if (leader) {
+        mma_rows_x_rows<D>(tmem + 0, q_desc, smem_desc_sw128(k_smem(s), 16, 1024));     // S
+        mma_rows_x_rows<D>(tmem + 128, do_desc, smem_desc_sw128(v_smem(s), 16, 1024));  // dP
+        tc_commit(s_full);
+      }
+      ok = wait(ds_full, jt & 1);
+      if (!ok) break;
+      tc_fence_after();
+      if (leader) {
+        // dQ += dS K_j (K_j read MN-major: the head dimension is contiguous)
+        mma_tmem_x_tile<D>(tmem + 256, tmem + 0,
+                           smem_desc_sw128(k_smem(s), L::kChunkBytes, 1024), jt > 0);
+        tc_commit(kv_empty(s));
+      }
+    }
+    if (leader) tc_commit(acc_done);
+    volatile int no_abort = 0;
+    mbar_wait(acc_done, 0, &no_abort, p.err, p.timeout_ns);
+  } else {
+    const int r = tid;
+    const int row = i * kBM + r;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tS = tmem + lane_base;
+    const uint32_t tP = tmem + lane_base + 128;
+    const size_t grow = static_cast<size_t>(bh) * p.Nq + row;
+    float lse2 = INFINITY, dl = 0.f;
+    if (row < p.Nq) {
+      lse2 = __ldg(p.lse + grow) * kLog2e;
+      dl = __ldg(p.delta + grow);
+    }
+    const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
+    const uint64_t nl2 = f2_pack(-lse2, -lse2);
+    bool ok = true;
+    for (int jt = 0; ok && jt < n_kt; ++jt) {
+      const bool got = mbar_wait(s_full, jt & 1, abort_flag, p.err, p.timeout_ns);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int kbase = jt * kBM;
+      const bool need_mask = (kbase + kBM > p.Nk) || (p.causal && kbase + kBM - 1 > i * kBM + off);
+      int lim = p.Nk - 1 - kbase;
+      if (p.causal) lim = min(lim, row + off - kbase);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sv[32], dv[32];
+        tmem_ld32(tS + 32 * c, sv);
+        tmem_ld32(tP + 32 * c, dv);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), c2, nl2),
+                    x0, x1);
+          float p0 = ex2(x0), p1 = ex2(x1);
+          if (need_mask) {
+            if (32 * c + e > lim) p0 = 0.f;
+            if (32 * c + e + 1 > lim) p1 = 0.f;
+          }
+          pk[e >> 1] = pack_bf16x2(p0 * (__uint_as_float(dv[e]) - dl),
+                                   p1 * (__uint_as_float(dv[e + 1]) - dl));
+        }
+        tmem_st16(tS + 16 * c, pk);     // over columns already read
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(ds_full);
+    }
+    const bool fin = ok && (n_kt == 0 || mbar_wait(acc_done, 0, abort_flag, p.err, p.timeout_ns));
+    if (__all_sync(0xffffffffu, fin)) {
+      tc_fence_after();
+      uint16_t* dst = p.dq + grow * D;
+      if (n_kt == 0) {
+        if (row < p.Nq) store_zero_row<D>(dst);
+      } else {
+        store_row_bf16<D>(tmem + lane_base + 256, p.scale, dst, row < p.Nq);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// 3-D map over a contiguous [Z, N, D] bf16 tensor, box {64, 128, 1}, 128-byte swizzle.
+int encode_tile_map(CUtensorMap* m, const void* base, int D, int N, int Z) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(N),
+                            static_cast<uint64_t>(Z)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2,
+                               static_cast<uint64_t>(N) * static_cast<uint64_t>(D) * 2};
+  const uint32_t box[3] = {64, 128, 1};
+  return encode_tensor_map_16bit(m, base, true, 3, dims, strides, box);
+}
+
+template <int D>
+int launch_bwd_typed(const void* q, const void* k, const void* v, const void* o,
+                     const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                     float* delta, int B, int Hq, int Hkv, int Nq, int Nk, float scale,
+                     int causal, cudaStream_t stream, int device) {
+  using L = BwdLayout<D>;
+  static bool attr_done[64] = {};
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> g(mu);
+    if (device < 0 || device >= 64) return set_error(FA_ERR_CUDA, "device ordinal out of range");
+    if (!attr_done[device]) {
+      cudaError_t e = cudaFuncSetAttribute(fa_bwd_dkdv_kernel<D>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           L::kSmemBytes);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(fa_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 L::kSmemBytes);
+      if (e != cudaSuccess)
+        return set_error(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+      attr_done[device] = true;
+    }
+  }
+  BwdParams prm;
+  prm.o = static_cast<const uint16_t*>(o);
+  prm.dout = static_cast<const uint16_t*>(dout);
+  prm.lse = lse;
+  prm.delta = delta;
+  prm.dq = static_cast<uint16_t*>(dq);
+  prm.dk = static_cast<uint16_t*>(dk);
+  prm.dv = static_cast<uint16_t*>(dv);
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.Nq = Nq;
+  prm.Nk = Nk;
+  prm.causal = causal ? 1 : 0;
+  prm.scale = scale;
+  prm.scale_log2 = scale * kLog2e;
+  prm.err = device_error_word(device);
+  prm.timeout_ns = kWaitLimitNs;
+  if (!prm.err) return set_error(FA_ERR_CUDA, "device error word unavailable");
+
+  const long long rows = static_cast<long long>(B) * Hq * Nq;
+  int nsm = 0;
+  if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
+      nsm <= 0)
+    return set_error(FA_ERR_CUDA, "cannot read the SM count of device %d", device);
+  const int dgrid = static_cast<int>(std::min<long long>((rows + 7) / 8, 16LL * nsm));
+  if (dgrid > 0)
+    fa_bwd_delta_kernel<D><<<dgrid, 256, 0, stream>>>(prm.o, prm.dout, delta, rows);
+
+  // A side with no rows (Nq == 0: dK = dV = 0; Nk == 0: dQ = 0) gets a copy of
+  // the other side's maps, which its kernel then never reads.
+  CUtensorMap tq, tk, tv, tdo;
+  int rc;
+  if (Nq > 0) {
+    if ((rc = encode_tile_map(&tq, q, D, Nq, B * Hq)) != FA_OK) return rc;
+    if ((rc = encode_tile_map(&tdo, dout, D, Nq, B * Hq)) != FA_OK) return rc;
+  }
+  if (Nk > 0) {
+    if ((rc = encode_tile_map(&tk, k, D, Nk, B * Hkv)) != FA_OK) return rc;
+    if ((rc = encode_tile_map(&tv, v, D, Nk, B * Hkv)) != FA_OK) return rc;
+  }
+  if (Nq == 0 && Nk == 0) return FA_OK;
+  if (Nq == 0) {
+    tq = tk;
+    tdo = tk;
+  }
+  if (Nk == 0) {
+    tk = tq;
+    tv = tq;
+  }
+  const long long kv_ctas = static_cast<long long>(B) * Hkv * ((Nk + kBM - 1) / kBM);
+  const long long q_ctas = static_cast<long long>(B) * Hq * ((Nq + kBM - 1) / kBM);
+  if (kv_ctas > 0x7fffffffLL || q_ctas > 0x7fffffffLL)
+    return set_error(FA_ERR_UNSUPPORTED, "too many tiles");
+  if (kv_ctas > 0)
+    fa_bwd_dkdv_kernel<D><<<static_cast<unsigned>(kv_ctas), kThreads, L::kSmemBytes, stream>>>(
+        tq, tk, tv, tdo, prm);
+  if (q_ctas > 0)
+    fa_bwd_dq_kernel<D><<<static_cast<unsigned>(q_ctas), kThreads, L::kSmemBytes, stream>>>(
+        tq, tk, tv, tdo, prm);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(FA_ERR_CUDA, "fa_bwd launch: %s", cudaGetErrorString(e));
+  return FA_OK;
+}
+
+}  // namespace
+
+int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+               const void* dout, void* dq, void* dk, void* dv, float* delta, int B, int Hq,
+               int Hkv, int Nq, int Nk, int D, float scale, int causal, cudaStream_t stream,
+               int device) {
+  if (D == 128)
+    return launch_bwd_typed<128>(q, k, v, o, lse, dout, dq, dk, dv, delta, B, Hq, Hkv, Nq, Nk,
+                                 scale, causal, stream, device);
+  if (D == 64)
+    return launch_bwd_typed<64>(q, k, v, o, lse, dout, dq, dk, dv, delta, B, Hq, Hkv, Nq, Nk,
+                                scale, causal, stream, device);
+  return set_error(FA_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", D);
+}
+
+}  // namespace fa

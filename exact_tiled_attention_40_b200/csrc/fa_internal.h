@@ -73,6 +73,13 @@ int launch_merge_partials(float* o_acc, float* lse_acc, const void* o_part, cons
                           void* o_out, long long rows, int D, int first, cudaStream_t stream,
                           int device);
 
+// Attention backward with recomputation (validated arguments, bf16): delta
+// [B * Hq, Nq] fp32 is written (rowsum(dO * O)), then dK, dV and dQ.
+int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+               const void* dout, void* dq, void* dk, void* dv, float* delta, int B, int Hq,
+               int Hkv, int Nq, int Nk, int D, float scale, int causal, cudaStream_t stream,
+               int device);
+
 // Release cached per-device resources owned by the decode path.
 void release_decode_resources();
 

@@ -38,6 +38,7 @@ _SIGS = {
     "fa_quantize_e4m3": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P]),
     "fa_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_merge_partials": (_I, [_P, _P, _P, _P, _P, ctypes.c_longlong, _I, _I, _P]),
+    "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _I, _I, _P]),
     "fa_decode_paged_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _I, _I,
                                      _P]),
@@ -247,6 +248,34 @@ def attention_fp8(q, k, v, scale=None, causal=False, signs=None, return_lse=True
     k8, ks = quantize_e4m3(k, 128, signs)
     v8, vs = quantize_e4m3(v, 0)
     return attention_fp8_quantised(q8, k8, v8, qs, ks, vs, scale, causal, return_lse)
+
+
+def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, delta, B, Hq, Hkv, Nq, Nk, D, scale, causal,
+           stream=None):
+    """Raw call of the backward's C entry point."""
+    s = _stream(q.device) if stream is None else ctypes.c_void_p(stream)
+    _check(lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
+                        _ptr(dk), _ptr(dv), _ptr(delta), B, Hq, Hkv, Nq, Nk, D, float(scale),
+                        int(bool(causal)), s), "fa_bwd")
+
+
+def attention_backward(q, k, v, o, lse, dout, scale=None, causal=False):
+    """(dQ, dK, dV) bf16 of attention(q, k, v) for the output gradient dout, given the
+    forward's o and lse (q, o, dout [B,Hq,Nq,D]; k, v [B,Hkv,Nk,D]; bf16 CUDA)."""
+    for t in (q, k, v, o, lse, dout):
+        if not t.is_cuda:
+            raise FAError(1, "attention_backward", "tensors must live on a CUDA device")
+    if any(t.dtype != torch.bfloat16 for t in (q, k, v, o, dout)) or lse.dtype != torch.float32:
+        raise FAError(1, "attention_backward", "bf16 q, k, v, o, dout and fp32 lse expected")
+    q, k, v, o, dout, lse = (t.contiguous() for t in (q, k, v, o, dout, lse))
+    B, Hq, Nq, D = q.shape
+    _, Hkv, Nk, _ = k.shape
+    if scale is None:
+        scale = D ** -0.5
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    delta = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, delta, B, Hq, Hkv, Nq, Nk, D, scale, causal)
+    return dq, dk, dv
 
 
 def merge_partials(o_acc, lse_acc, o_part, lse_part, first=False, o_out=None, stream=None):

@@ -185,6 +185,26 @@ int fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_sc
                int Hkv, int Nq, int Nk, int D, float scale, int causal, fa_stream_t stream);
 
 /*
+ * Backward pass of fa_fwd (bf16) with recomputation: unite.ai page above, which
+ * names recomputation (P is not stored; it is rebuilt tile by tile from the
+ * saved LSE).  With P = exp(scale Q K^T - LSE) (causal: bottom-right mask) and
+ * delta_i = sum_d dO_id O_id:
+ *     dV = P^T dO,  dS = P * (dO V^T - delta),  dQ = scale dS K,  dK = scale dS^T Q;
+ * the query heads of a KV head add into its dK and dV (GQA).
+ *   q, o, dout [B, Hq, Nq, D] bf16; k, v [B, Hkv, Nk, D] bf16
+ *   lse        [B, Hq, Nq] fp32 (fa_fwd's LSE for the same inputs)
+ *   dq         [B, Hq, Nq, D] bf16 (written); dk, dv [B, Hkv, Nk, D] bf16 (written)
+ *   delta      [B, Hq, Nq] fp32 (written: rowsum(dout * o), caller-provided scratch)
+ * Rules of fa_fwd for sizes, GQA, causal and alignment; D in {64, 128}.  Keys
+ * that no query sees get dK = dV = 0.  Three kernels, no atomics, nothing
+ * allocated: rows of delta, then dK/dV (a CTA per key tile), then dQ (a CTA per
+ * query tile); P and dS are rounded to bf16 before their tensor-core products.
+ */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dout, void* dq, void* dk, void* dv, float* delta, int B, int Hq, int Hkv,
+           int Nq, int Nk, int D, float scale, int causal, fa_stream_t stream);
+
+/*
  * Merge of partial attention results over disjoint key sets (the combine step
  * of the split-KV decode, exposed for sequence-sharded prefill: each rank's
  * queries meet the K/V chunks of every rank and fold each chunk's result in).

@@ -219,3 +219,33 @@ def test_merge_rejects_bad_arguments_on_the_host(lib, kw, code):
 
 def test_merge_of_no_rows_is_a_noop(lib):
     assert merge(lib, rows=0, oa=None, op=None) == 0
+
+
+def bwd(lib, B=1, Hq=2, Hkv=1, Nq=8, Nk=8, D=128, scale=0.1, causal=0, q=FAKE, k=FAKE, v=FAKE,
+        o=FAKE, lse=FAKE, do=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, delta=FAKE):
+    return lib.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, delta, B, Hq, Hkv, Nq, Nk, D, scale,
+                      causal, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=-1), "FA_ERR_INVALID_ARG"),
+    (dict(D=96), "FA_ERR_UNSUPPORTED"),
+    (dict(Hq=3, Hkv=2), "FA_ERR_INVALID_ARG"),
+    (dict(causal=1, Nq=9, Nk=8), "FA_ERR_INVALID_ARG"),
+    (dict(scale=0.0), "FA_ERR_INVALID_ARG"),
+    (dict(lse=None), "FA_ERR_INVALID_ARG"),
+    (dict(delta=None), "FA_ERR_INVALID_ARG"),
+    (dict(dk=None), "FA_ERR_INVALID_ARG"),
+    (dict(do=FAKE + 2), "FA_ERR_INVALID_ARG"),
+    (dict(dv=FAKE + 8), "FA_ERR_INVALID_ARG"),
+])
+def test_bwd_rejects_bad_arguments_on_the_host(lib, kw, code):
+    assert bwd(lib, **kw) == E[code]
+
+
+def test_bwd_empty_problems(lib):
+    assert bwd(lib, B=0) == 0
+    assert bwd(lib, Nq=0, Nk=0) == 0
+    # no queries but keys: dK = dV = 0 must still be written, so the call reaches the device
+    assert bwd(lib, Nq=0, q=None, o=None, lse=None, do=None, dq=None, delta=None) in (
+        0, E["FA_ERR_NO_DEVICE"])
