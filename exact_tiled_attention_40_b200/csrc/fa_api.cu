@@ -40,6 +40,19 @@ int* device_error_word(int device) {
   return g_err_ptr[device];
 }
 
+int device_sm_count(int device) {
+  static int cached[64] = {};
+  static std::mutex mu;
+  std::lock_guard<std::mutex> g(mu);
+  if (device < 0 || device >= 64) return 0;
+  if (!cached[device]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) n = 0;
+    cached[device] = n;
+  }
+  return cached[device];
+}
+
 namespace {
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,

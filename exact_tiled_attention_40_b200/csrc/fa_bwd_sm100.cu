@@ -640,10 +640,8 @@ int launch_bwd_typed(const void* q, const void* k, const void* v, const void* o,
   if (!prm.err) return set_error(FA_ERR_CUDA, "device error word unavailable");
 
   const long long rows = static_cast<long long>(B) * Hq * Nq;
-  int nsm = 0;
-  if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
-      nsm <= 0)
-    return set_error(FA_ERR_CUDA, "cannot read the SM count of device %d", device);
+  const int nsm = device_sm_count(device);
+  if (nsm <= 0) return set_error(FA_ERR_CUDA, "cannot read the SM count of device %d", device);
   const int dgrid = static_cast<int>(std::min<long long>((rows + 7) / 8, 16LL * nsm));
   if (dgrid > 0)
     fa_bwd_delta_kernel<D><<<dgrid, 256, 0, stream>>>(prm.o, prm.dout, delta, rows);

@@ -648,19 +648,6 @@ int encode_codes(CUtensorMap* m, const void* base, int N, int Z) {
   return encode_tensor_map_u8(m, base, 3, dims, strides, box);
 }
 
-int sm_count(int device) {
-  static int cached[64] = {};
-  static std::mutex mu;
-  std::lock_guard<std::mutex> g(mu);
-  if (device < 0 || device >= 64) return 0;
-  if (!cached[device]) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) n = 0;
-    cached[device] = n;
-  }
-  return cached[device];
-}
-
 }  // namespace
 
 int launch_quantize_e4m3(const void* x, void* codes, float* scales, int Z, int N, int D,
@@ -728,7 +715,7 @@ int launch_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* 
   const long long items = static_cast<long long>(prm.num_mpairs) * B * Hq;
   if (items > 0x7fffffffLL) return set_error(FA_ERR_UNSUPPORTED, "too many work items");
   prm.num_items = static_cast<int>(items);
-  const int nsm = sm_count(device);
+  const int nsm = device_sm_count(device);
   if (nsm <= 0) return set_error(FA_ERR_CUDA, "cannot read the SM count of device %d", device);
   const int grid = static_cast<int>(std::min<long long>(items, nsm));
   if (grid == 0) return FA_OK;

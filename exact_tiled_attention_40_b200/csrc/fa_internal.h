@@ -25,6 +25,9 @@ int encode_tensor_map_16bit(CUtensorMap* m, const void* base, bool bf16, int ran
 int encode_tensor_map_u8(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
                          const uint64_t* strides_bytes, const uint32_t* box);
 
+// Number of SMs of `device` (cached per device), 0 if it cannot be read.
+int device_sm_count(int device);
+
 // Wall-time limit of every bounded wait inside a kernel.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 

@@ -108,10 +108,8 @@ __global__ void __launch_bounds__(kMergeThreads)
 int launch_merge_partials(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
                           void* o_out, long long rows, int D, int first, cudaStream_t stream,
                           int device) {
-  int nsm = 0;
-  if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
-      nsm <= 0)
-    return set_error(FA_ERR_CUDA, "cannot read the SM count of device %d", device);
+  const int nsm = device_sm_count(device);
+  if (nsm <= 0) return set_error(FA_ERR_CUDA, "cannot read the SM count of device %d", device);
   const long long per_block = kMergeThreads / 32;
   const long long want = (rows + per_block - 1) / per_block;
   const int grid = static_cast<int>(std::min<long long>(want, 8LL * nsm));

@@ -2,6 +2,15 @@
 
     python -m exact_tiled_attention_40_b200.run_case --case gqa_b1_hq32_hkv8_n8192_d128_causal
     python -m exact_tiled_attention_40_b200.run_case --case decode_b64_hq32_hkv8_d128_page16
+    python -m exact_tiled_attention_40_b200.run_case --case gqa_b1_hq32_hkv8_n8192_d128_causal --op bwd
+    python -m exact_tiled_attention_40_b200.run_case --case fp8_gqa_b1_hq32_hkv8_n8192_d128_causal
+    python -m exact_tiled_attention_40_b200.run_case --case fp8_gqa_b1_hq32_hkv8_n8192_d128_causal --op quantize
+
+--op bwd times fa_bwd on a prefill case (its inputs: the library forward's O and
+LSE and a seeded output gradient); its rate counts the backward's five matrix
+products, 2.5 times the forward's FLOPs.  For an FP8 case the inputs are
+quantised once before timing and fa_fwd_fp8 is timed (--op quantize times
+fa_quantize_e4m3 of Q, K and V instead, in GB/s of bf16 read and codes written).
 
 Inputs come from the seeded generator and stay resident on the device; a
 256 MiB buffer is written before every launch so no launch finds its inputs in
@@ -17,21 +26,60 @@ import statistics
 import torch
 
 from . import fa
-from .inputs import (DECODE_CASES, PAGED_PREFILL_CASES, PREFILL_CASES, VARLEN_CASES,
-                     make_decode, make_paged_prefill, make_prefill, make_varlen, varlen_flops)
+from .inputs import (DECODE_CASES, FP8_CASES, PAGED_PREFILL_CASES, PREFILL_CASES, VARLEN_CASES,
+                     hadamard_signs, make_decode, make_paged_prefill, make_prefill, make_varlen,
+                     varlen_flops)
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--case", required=True,
                     choices=sorted(PREFILL_CASES) + sorted(DECODE_CASES) + sorted(VARLEN_CASES)
-                    + sorted(PAGED_PREFILL_CASES))
+                    + sorted(PAGED_PREFILL_CASES) + sorted(FP8_CASES))
+    ap.add_argument("--op", default="fwd", choices=["fwd", "bwd", "quantize"])
     ap.add_argument("--iters", type=int, default=5)
     args = ap.parse_args()
     dev = torch.device("cuda", 0)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    if args.case in PREFILL_CASES:
+    if args.op == "bwd":
+        c = PREFILL_CASES[args.case]
+        q, k, v, gen = make_prefill(c)
+        do = torch.randn((c.B, c.Hq, c.Nq, c.D), generator=gen).to(torch.bfloat16)
+        q, k, v, do = q.to(dev), k.to(dev), v.to(dev), do.to(dev)
+        o, lse = fa.attention(q, k, v, c.softmax_scale, c.causal)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        delta = torch.empty((c.B, c.Hq, c.Nq), dtype=torch.float32, device=dev)
+
+        def launch():
+            fa.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, delta, c.B, c.Hq, c.Hkv, c.Nq, c.Nk, c.D,
+                      c.softmax_scale, c.causal, stream=stream.cuda_stream)
+        work, unit = 2.5 * c.flops / 1e12, "TFLOP/s"
+    elif args.case in FP8_CASES:
+        f = FP8_CASES[args.case]
+        c = f.prefill
+        q, k, v, _ = make_prefill(c)
+        q, k, v = q.to(dev), k.to(dev), v.to(dev)
+        signs = None if f.sign_seed is None else hadamard_signs(c.D, f.sign_seed).to(dev)
+        q8, qs = fa.quantize_e4m3(q, 128, signs)
+        k8, ks = fa.quantize_e4m3(k, 128, signs)
+        v8, vs = fa.quantize_e4m3(v, 0)
+        o = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((c.B, c.Hq, c.Nq), dtype=torch.float32, device=dev)
+        if args.op == "quantize":
+            def launch():
+                s_ = stream.cuda_stream
+                fa.fa_quantize_e4m3(q, q8, qs, c.B * c.Hq, c.Nq, c.D, 128, signs, stream=s_)
+                fa.fa_quantize_e4m3(k, k8, ks, c.B * c.Hkv, c.Nk, c.D, 128, signs, stream=s_)
+                fa.fa_quantize_e4m3(v, v8, vs, c.B * c.Hkv, c.Nk, c.D, 0, None, stream=s_)
+            elems = q.numel() + k.numel() + v.numel()
+            work, unit = 3 * elems / 1e9, "GB/s"
+        else:
+            def launch():
+                fa.fa_fwd_fp8(q8, k8, v8, qs, ks, vs, o, lse, c.B, c.Hq, c.Hkv, c.Nq, c.Nk, c.D,
+                              c.softmax_scale, c.causal, stream=stream.cuda_stream)
+            work, unit = c.flops / 1e12, "TFLOP/s"
+    elif args.case in PREFILL_CASES:
         c = PREFILL_CASES[args.case]
         q, k, v, _ = make_prefill(c)
         q, k, v = q.to(dev), k.to(dev), v.to(dev)
