@@ -3,13 +3,14 @@
 Inputs: q, k, v and the output gradient dO drawn by the shared generators; o
 and lse are the oracle forward's (o rounded to bf16, lse to fp32), and the
 oracle backward reads the same rounded values.  Tolerance, derived from the
-kernel's arithmetic: P and dS are rounded to bf16 before their tensor-core
-products (relative 2^-9 each), every output is rounded to bf16 (2^-9 of the
-result, itself at most the sum of its terms' magnitudes), and the fp32
-recomputation of P costs < 1e-4 relative.  So for every element
-    |d dV_jd| <= (2^-8 + 1e-4) sum_i P_ij |dO_id|,
-    |d dK_jd| <= (2^-8 + 1e-4) scale sum_i |dS_ij| |Q_id|,
-    |d dQ_id| <= (2^-8 + 1e-4) scale sum_j |dS_ij| |K_jd|,
+kernel's arithmetic (bf16 keeps 8 significant bits: rounding to nearest is
+within 2^-8 relative): P and dS are rounded to bf16 before their tensor-core
+products (2^-8 each), every output is rounded to bf16 (2^-8 of the result,
+itself at most the sum of its terms' magnitudes), and the fp32 recomputation of
+P costs < 1e-4 relative.  So for every element
+    |d dV_jd| <= (2^-7 + 1e-4) sum_i P_ij |dO_id|,
+    |d dK_jd| <= (2^-7 + 1e-4) scale sum_i |dS_ij| |Q_id|,
+    |d dQ_id| <= (2^-7 + 1e-4) scale sum_j |dS_ij| |K_jd|,
 plus 1e-6 (summed over the query heads of a KV head for dK, dV).
 
 These tests wait for their first run on a B200: they run when the environment
@@ -29,7 +30,7 @@ pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not os.environ.get("FA_PENDING_GPU_TESTS"),
                                  reason="awaiting a first B200 run: FA_PENDING_GPU_TESTS")]
 
-U = 2.0 ** -8 + 1e-4
+U = 2.0 ** -7 + 1e-4
 
 
 def f64(t):
