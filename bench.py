@@ -307,6 +307,82 @@ def widened_rows(fa, dev, stream, flush, warmup, steps, peaks, peak_src):
     return out
 
 
+def pending_rows(fa, dev, stream, flush, warmup, steps, peaks, peak_src):
+    """Kernels built but not yet verified on a B200 (FP8 forward and its
+    quantiser, backward): timed on the headline prefill workload only when
+    --pending is given, never in a default run."""
+    from exact_tiled_attention_40_b200.inputs import FP8_CASES, hadamard_signs
+    out = {}
+    sp = stream.cuda_stream
+
+    def timed(launch):
+        ts = []
+        for i in range(warmup + steps):
+            flush.fill_(i & 0xff)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            launch()
+            b.record(stream)
+            b.synchronize()
+            if i >= warmup:
+                ts.append(a.elapsed_time(b))
+        if fa.device_status() != 0:
+            raise RuntimeError(fa.last_error())
+        return statistics.median(ts)
+
+    f = FP8_CASES["fp8_gqa_b1_hq32_hkv8_n8192_d128_causal"]
+    c = f.prefill
+    try:
+        q_h, k_h, v_h, gen = make_prefill(c)
+        q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+        signs = hadamard_signs(c.D, f.sign_seed).to(dev)
+        q8, qs = fa.quantize_e4m3(q, 128, signs)
+        k8, ks = fa.quantize_e4m3(k, 128, signs)
+        v8, vs = fa.quantize_e4m3(v, 0)
+        o = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((c.B, c.Hq, c.Nq), dtype=torch.float32, device=dev)
+
+        def quant():
+            fa.fa_quantize_e4m3(q, q8, qs, c.B * c.Hq, c.Nq, c.D, 128, signs, stream=sp)
+            fa.fa_quantize_e4m3(k, k8, ks, c.B * c.Hkv, c.Nk, c.D, 128, signs, stream=sp)
+            fa.fa_quantize_e4m3(v, v8, vs, c.B * c.Hkv, c.Nk, c.D, 0, None, stream=sp)
+        ms = timed(quant)
+        gbs = 3 * (q.numel() + k.numel() + v.numel()) / (ms * 1e-3) / 1e9
+        out["quantize_e4m3"] = {"workload": f.name, "value": gbs, "unit": "GB/s",
+                                "ms_per_launch": ms,
+                                "roofline": {"bound": "hbm", "achieved": gbs,
+                                             "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                             "frac": gbs / peaks["hbm_gbs"],
+                                             "peak_source": f"{peak_src} copy"}}
+        ms = timed(lambda: fa.fa_fwd_fp8(q8, k8, v8, qs, ks, vs, o, lse, c.B, c.Hq, c.Hkv, c.Nq,
+                                         c.Nk, c.D, c.softmax_scale, c.causal, stream=sp))
+        tf = c.flops / (ms * 1e-3) / 1e12
+        pk = 2 * peaks["bf16_tflops"]
+        out["fp8_prefill"] = {"workload": f.name, "value": tf, "unit": "TFLOP/s",
+                              "ms_per_launch": ms,
+                              "roofline": {"bound": "tensor", "achieved": tf, "peak": pk,
+                                           "unit": "TFLOP/s", "frac": tf / pk,
+                                           "peak_source": f"{peak_src} burst bf16 x 2 "
+                                                          "(nominal fp8 / bf16 ratio)"}}
+        do = torch.randn(q.shape, generator=gen).to(torch.bfloat16).to(dev)
+        ob, lb = fa.attention(q, k, v, c.softmax_scale, c.causal)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        delta = torch.empty((c.B, c.Hq, c.Nq), dtype=torch.float32, device=dev)
+        ms = timed(lambda: fa.fa_bwd(q, k, v, ob, lb, do, dq, dk, dv, delta, c.B, c.Hq, c.Hkv,
+                                     c.Nq, c.Nk, c.D, c.softmax_scale, c.causal, stream=sp))
+        tf = 2.5 * c.flops / (ms * 1e-3) / 1e12
+        out["backward"] = {"workload": c.name, "value": tf, "unit": "TFLOP/s",
+                           "ms_per_launch": ms, "flops": "2.5 x the forward's",
+                           "roofline": {"bound": "tensor", "achieved": tf,
+                                        "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                        "frac": tf / peaks["bf16_tflops"],
+                                        "peak_source": f"{peak_src} burst bf16"}}
+    except Exception as e:  # reported, never fatal for the headline line
+        out["error"] = f"{type(e).__name__}: {e}"[:300]
+    return out
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return 0
@@ -343,6 +419,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pending", action="store_true",
+                    help="also time the kernels that await their first B200 verification")
     args = ap.parse_args()
     world, rank, local = dist_env()
     if args.impl == "reference":
@@ -503,6 +581,9 @@ def main():
                                 "kind": "oracle", "sample": sample, "seconds": dt}
         # rows beyond the headline path, measured outside its timed region
         line["widened"] = widened_rows(fa, dev, stream, flush, args.warmup, min(args.steps, 10),
+                                       peaks, peak_src)
+    if rank == 0 and world == 1 and args.pending:
+        line["pending"] = pending_rows(fa, dev, stream, flush, args.warmup, min(args.steps, 10),
                                        peaks, peak_src)
     if rank == 0:
         print(json.dumps(line), flush=True)
