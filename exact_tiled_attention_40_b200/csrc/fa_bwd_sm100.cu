@@ -56,7 +56,10 @@ struct BwdLayout {
   static constexpr int kBarOff = kRingOff + 4 * kTileBytes;
   static constexpr int kNumBars = 1 + 2 + 2 + 1 + 1 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
+  // at least 118 KB so that two CTAs never share an SM: each allocates all 512
+  // TMEM columns (the next power of two above its 384 or 320 at D = 64)
+  static constexpr int kSmemBytes =
+      (kMiscOff + 16 + 1024) > 118 * 1024 ? (kMiscOff + 16 + 1024) : 118 * 1024;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
