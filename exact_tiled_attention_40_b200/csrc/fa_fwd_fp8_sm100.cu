@@ -209,6 +209,13 @@ constexpr int kSlots = 10;          // K/V ring slots
 constexpr float kTau = 0.5f;        // lazy-rescale threshold (log2 units)
 constexpr float kPOff = 8.f;        // p = 2^(x - m_ref + kPOff)
 constexpr int kThreads = 384;
+#ifndef FA_FP8_HALF_EXP
+#define FA_FP8_HALF_EXP 0
+#endif
+// 1: the exponentials of P in f16 pairs (ex2.approx.f16x2), converted straight
+// to E4M3; 0: one fp32 exponential per element.
+constexpr bool kHalfExp = FA_FP8_HALF_EXP != 0;
+constexpr uint32_t kF16x2Off = 0x5C005C00u;   // (256, 256) in f16: 2^kPOff
 constexpr uint32_t kRegsControl = 72;
 constexpr uint32_t kRegsSoftmax = 216;
 static_assert(kRegsControl * 128 + kRegsSoftmax * 256 <= 384 * 168, "register split");
@@ -564,7 +571,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st32(tO + 32 * cc, ov);
           }
         }
-        const float neg_m = (m_used == -INFINITY) ? 0.f : kPOff - m_used;
+        // the half-precision variant exponentiates x - m_ref (small for the
+        // entries that matter, so f16 keeps them accurate) and applies the
+        // 2^kPOff offset as an exact f16 product; its L then has no offset
+        const float neg_m = (m_used == -INFINITY) ? 0.f : (kHalfExp ? 0.f : kPOff) - m_used;
         const uint64_t c2 = f2_pack(c, c);
         const uint64_t nm2 = f2_pack(neg_m, neg_m);
         uint64_t sum2[4] = {0, 0, 0, 0};
@@ -579,9 +589,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                              nm2), x0, x1);
             f2_unpack(f2_fma(f2_pack(__uint_as_float(s[k0 + 2]), __uint_as_float(s[k0 + 3])), c2,
                              nm2), x2, x3);
-            const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
-            sum2[e & 3] = f2_add(sum2[e & 3], f2_add(f2_pack(p0, p1), f2_pack(p2, p3)));
-            pk[e] = pack_e4m3x4(p0, p1, p2, p3);
+            if constexpr (kHalfExp) {
+              // exponent pairs in f16, two exponentials per MUFU instruction
+              const uint32_t h01 = ex2_f16x2(pack_f16x2(x0, x1));
+              const uint32_t h23 = ex2_f16x2(pack_f16x2(x2, x3));
+              float p0, p1, p2, p3;
+              unpack_f16x2(h01, p0, p1);
+              unpack_f16x2(h23, p2, p3);
+              sum2[e & 3] = f2_add(sum2[e & 3], f2_add(f2_pack(p0, p1), f2_pack(p2, p3)));
+              pk[e] = static_cast<uint32_t>(e4m3x2_from_f16x2(mul_f16x2(h01, kF16x2Off))) |
+                      (static_cast<uint32_t>(e4m3x2_from_f16x2(mul_f16x2(h23, kF16x2Off)))
+                       << 16);
+            } else {
+              const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+              sum2[e & 3] = f2_add(sum2[e & 3], f2_add(f2_pack(p0, p1), f2_pack(p2, p3)));
+              pk[e] = pack_e4m3x4(p0, p1, p2, p3);
+            }
           }
           tmem_st8(tS + 8 * cq, pk);
           if (cq == 1) {                           // keys 0-63 of P are in place
@@ -604,7 +627,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = false;
       } else {
         tc_fence_after();
-        const float inv = l > 0.f ? v_s / l : 0.f;
+        const float l_p = kHalfExp ? l * 256.f : l;   // the sum of the p that P holds
+        const float inv = l > 0.f ? v_s / l_p : 0.f;
 #pragma unroll 1
         for (int cc = 0; cc < kD / 32; ++cc) {
           uint32_t ov[32];
@@ -624,7 +648,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (p.lse && row < p.Nq)
           p.lse[row_index] =
-              l > 0.f ? (m_used - kPOff + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+              l > 0.f ? (m_used - (kHalfExp ? 0.f : kPOff) + __log2f(l)) * 0.69314718055994530942f
+                      : -INFINITY;
       }
     }
   }

@@ -371,6 +371,32 @@ __device__ __forceinline__ uint16_t pack_e4m3x2(float a, float b) {
   return r;
 }
 
+// Two base-2 exponentials of an f16 pair (MUFU, approximate).
+__device__ __forceinline__ uint32_t ex2_f16x2(uint32_t x) {
+  uint32_t y;
+  asm("ex2.approx.f16x2 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+// f16 pair (lo in bits 0-15) -> E4M3 pair (lo in bits 0-7), nearest even, saturating.
+__device__ __forceinline__ uint16_t e4m3x2_from_f16x2(uint32_t h) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(r) : "r"(h));
+  return r;
+}
+// Product of two f16 pairs (round to nearest).
+__device__ __forceinline__ uint32_t mul_f16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+// f16 pair -> two fp32 (exact).
+__device__ __forceinline__ void unpack_f16x2(uint32_t h, float& lo, float& hi) {
+  asm("{\n\t.reg .f16 l, u;\n\tmov.b32 {l, u}, %2;\n\t"
+      "cvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, u;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(h));
+}
+
 // ------------------------------------------------------------------ packed fp32 pairs
 // sm_100 executes fp32 add/mul/fma on register pairs in one instruction.
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
