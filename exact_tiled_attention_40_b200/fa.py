@@ -230,6 +230,13 @@ def attention_fp8_quantised(q8, k8, v8, q_scale, k_scale, v_scale, scale=None, c
         raise FAError(1, "attention_fp8", "codes must be uint8")
     B, Hq, Nq, D = q8.shape
     _, Hkv, Nk, _ = k8.shape
+    if k8.shape != v8.shape or k8.shape[0] != B or k8.shape[3] != D:
+        raise FAError(1, "attention_fp8", "k8, v8 must be [B, Hkv, Nk, D] like q8's B and D")
+    want = {"q_scale": (q_scale, B * Hq * (-(-Nq // 128))),
+            "k_scale": (k_scale, B * Hkv * (-(-Nk // 128))), "v_scale": (v_scale, B * Hkv)}
+    for name, (t, n) in want.items():
+        if t.dtype != torch.float32 or t.numel() != n:
+            raise FAError(1, "attention_fp8", f"{name} must hold {n} fp32 scales")
     if scale is None:
         scale = D ** -0.5
     o = torch.empty((B, Hq, Nq, D), dtype=torch.bfloat16, device=q8.device)

@@ -120,6 +120,10 @@ def ring_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bo
     one device.
     """
     import torch.distributed as dist
+    if q.dim() != 5 or k.dim() != 5 or q.shape[0] != 2 or k.shape != v.shape or \
+            k.shape[0] != 2 or k.shape[1] != q.shape[1] or k.shape[3:] != q.shape[3:]:
+        raise ValueError("q [2, B, Hq, C, D] and k, v [2, B, Hkv, C, D] expected "
+                         "(zigzag_shard of [B, H, N, D] tensors)")
     attend = attend or _default_attend
     merge = merge or _default_merge
     D = q.shape[-1]

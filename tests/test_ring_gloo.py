@@ -172,3 +172,13 @@ def test_one_rank_at_a_time_with_fetched_chunks_equals_the_oracle():
     np.testing.assert_allclose(ring.zigzag_unshard(outs).double().numpy(), O_ref, atol=2e-6)
     np.testing.assert_allclose(ring.zigzag_unshard(lses, dim=-1).double().numpy(), L_ref,
                                atol=2e-6)
+
+
+def test_ring_rejects_tensors_that_are_not_zigzag_shards():
+    q = torch.zeros((2, 1, 2, 8, 4))
+    k = torch.zeros((2, 1, 1, 8, 4))
+    with pytest.raises(ValueError):
+        ring.ring_attention(q[0], k, k, True, attend=_oracle_attend, merge=_oracle_merge)
+    with pytest.raises(ValueError):
+        ring.ring_attention(q, k[:, :, :, :4], k[:, :, :, :4], True, attend=_oracle_attend,
+                            merge=_oracle_merge)
