@@ -243,6 +243,23 @@ int paged_common(const void* q, const void* kcache, const void* vcache,
                     max_pages_per_seq * 16, D, scale, causal, bf16, stream, dev);
 }
 
+int fwd_host_common(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                    float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
+                    float* lse_dev, int B, int Hq, int Hkv, int Nq, int Nk, int D, float scale,
+                    int causal, cudaStream_t stream) {
+  int rc = validate_fwd(q_dev, k_dev, v_dev, o_dev, B, Hq, Hkv, Nq, Nk, D, scale, causal);
+  if (rc != FA_OK) return rc;
+  if (B == 0 || Hq == 0 || Nq == 0) return FA_OK;
+  if (!q_host || !o_host || (Nk > 0 && (!k_host || !v_host)))
+    return set_error(FA_ERR_INVALID_ARG, "null host pointer");
+  if ((lse_host == nullptr) != (lse_dev == nullptr))
+    return set_error(FA_ERR_INVALID_ARG, "lse_host and lse_dev must both be given or both NULL");
+  int dev;
+  if ((rc = current_sm100(&dev)) != FA_OK) return rc;
+  return launch_fwd_host(q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev, v_dev, o_dev,
+                         lse_dev, B, Hq, Hkv, Nq, Nk, D, scale, causal, stream, dev);
+}
+
 int quantize_common(const void* x, void* codes, float* scales, int Z, int N, int D,
                     int group_rows, const float* signs, cudaStream_t stream) {
   if (Z < 0 || N < 0) return set_error(FA_ERR_INVALID_ARG, "negative size");
@@ -340,6 +357,15 @@ int fa_merge_partials(float* o_acc, float* lse_acc, const void* o_part, const fl
                       void* o_out, long long rows, int D, int first, fa_stream_t stream) {
   return fa::merge_common(o_acc, lse_acc, o_part, lse_part, o_out, rows, D, first,
                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fa_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
+                float* lse_dev, int B, int Hq, int Hkv, int Nq, int Nk, int D, float scale,
+                int causal, fa_stream_t stream) {
+  return fa::fwd_host_common(q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev, v_dev, o_dev,
+                             lse_dev, B, Hq, Hkv, Nq, Nk, D, scale, causal,
+                             reinterpret_cast<cudaStream_t>(stream));
 }
 
 int fa_quantize_e4m3(const void* x, void* codes, float* scales, int Z, int N, int D,
@@ -488,7 +514,10 @@ int fa_device_status(void) {
                    word);
 }
 
-void fa_release(void) { fa::release_decode_resources(); }
+void fa_release(void) {
+  fa::release_decode_resources();
+  fa::release_host_pipeline_resources();
+}
 
 int fa_version(void) { return 100; }
 

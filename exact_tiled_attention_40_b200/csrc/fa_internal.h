@@ -83,6 +83,14 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
                int Hkv, int Nq, int Nk, int D, float scale, int causal, cudaStream_t stream,
                int device);
 
+// fa_fwd (bf16) from host buffers through caller-owned device buffers, the
+// copies of one chunk overlapping the forward of another (validated arguments).
+int launch_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                    float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
+                    float* lse_dev, int B, int Hq, int Hkv, int Nq, int Nk, int D, float scale,
+                    int causal, cudaStream_t stream, int device);
+void release_host_pipeline_resources();
+
 // Release cached per-device resources owned by the decode path.
 void release_decode_resources();
 

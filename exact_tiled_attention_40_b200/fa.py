@@ -35,6 +35,8 @@ _SIGS = {
                                 _I, _P]),
     "fa_fwd_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I,
                           _F, _I, _P]),
+    "fa_fwd_host": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I,
+                         _P]),
     "fa_quantize_e4m3": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P]),
     "fa_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_merge_partials": (_I, [_P, _P, _P, _P, _P, ctypes.c_longlong, _I, _I, _P]),
@@ -180,6 +182,45 @@ def prefill_paged(q, kcache, vcache, block_table, cu_seqlens_q, seq_lens_k, max_
                  int(max_seqlen_q), block_table.shape[1], num_pages, total_q, D, page_size, scale,
                  causal)
     return o, lse
+
+
+def fa_fwd_host(q_host, k_host, v_host, o_host, lse_host, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk,
+                D, scale, causal, stream=None):
+    """Raw call of the host-buffer forward (bf16): *_host are CPU tensors, the others
+    the device staging tensors of the same shapes."""
+    s = _stream(q.device) if stream is None else ctypes.c_void_p(stream)
+    _check(lib().fa_fwd_host(_ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(o_host),
+                             _ptr(lse_host), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq,
+                             Hkv, Nq, Nk, D, float(scale), int(bool(causal)), s), "fa_fwd_host")
+
+
+def attention_from_host(q_host, k_host, v_host, scale=None, causal=False, device=None,
+                        staging=None):
+    """O and LSE in pinned host memory for bf16 q_host [B,Hq,Nq,D], k_host, v_host
+    [B,Hkv,Nk,D] (contiguous, preferably pinned CPU tensors); the copies overlap the
+    forward chunk by chunk.  `staging` = (q, k, v, o, lse) device tensors to reuse.
+    Asynchronous like every call here: the host outputs are complete once the
+    current stream has passed this call (e.g. after torch.cuda.synchronize())."""
+    for t in (q_host, k_host, v_host):
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise FAError(1, "attention_from_host", "contiguous bf16 CPU tensors expected")
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    B, Hq, Nq, D = q_host.shape
+    _, Hkv, Nk, _ = k_host.shape
+    if scale is None:
+        scale = D ** -0.5
+    if staging is None:
+        staging = (torch.empty(q_host.shape, dtype=torch.bfloat16, device=device),
+                   torch.empty(k_host.shape, dtype=torch.bfloat16, device=device),
+                   torch.empty(v_host.shape, dtype=torch.bfloat16, device=device),
+                   torch.empty(q_host.shape, dtype=torch.bfloat16, device=device),
+                   torch.empty((B, Hq, Nq), dtype=torch.float32, device=device))
+    o_host = torch.empty(q_host.shape, dtype=torch.bfloat16, pin_memory=True)
+    lse_host = torch.empty((B, Hq, Nq), dtype=torch.float32, pin_memory=True)
+    q, k, v, o, lse = staging
+    fa_fwd_host(q_host, k_host, v_host, o_host, lse_host, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, D,
+                scale, causal)
+    return o_host, lse_host
 
 
 def fa_quantize_e4m3(x, codes, scales, Z, N, D, group_rows, signs=None, stream=None):

@@ -137,6 +137,25 @@ int fa_fwd_paged(const void* q, const void* kcache, const void* vcache,
                  float scale, int causal, fa_stream_t stream);
 
 /*
+ * fa_fwd (bf16) with the inputs in HOST memory and the outputs wanted there.
+ *   q_host, k_host, v_host, o_host, lse_host: host buffers with fa_fwd's layouts
+ *     (page-locked for the copies to run asynchronously and overlap)
+ *   q_dev, k_dev, v_dev, o_dev, lse_dev: device buffers of the same sizes, owned
+ *     by the caller, used as staging (their contents are overwritten)
+ *   lse_host and lse_dev are both given or both NULL.
+ * The work is cut into about eight chunks (whole sequences, or whole GQA groups
+ * of a sequence); each chunk's inputs are copied in while the previous chunk is
+ * computed and the one before it copied out, on two library-owned copy streams
+ * ordered against `stream` by events: the call is asynchronous on `stream` like
+ * fa_fwd, and the host outputs are complete once `stream` reaches the point of
+ * the call.  fa_release() destroys the copy streams.  Argument rules as fa_fwd.
+ */
+int fa_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
+                float* lse_dev, int B, int Hq, int Hkv, int Nq, int Nk, int D, float scale,
+                int causal, fa_stream_t stream);
+
+/*
  * E4M3 (FP8) quantisation of a bf16 tensor, the input preparation of
  * fa_fwd_fp8.  unite.ai, "Flash Attention: Revolutionizing Transformer
  * Efficiency", section "Flash Attention-3", names FP8 inputs with block

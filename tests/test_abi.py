@@ -249,3 +249,28 @@ def test_bwd_empty_problems(lib):
     # no queries but keys: dK = dV = 0 must still be written, so the call reaches the device
     assert bwd(lib, Nq=0, q=None, o=None, lse=None, do=None, dq=None, delta=None) in (
         0, E["FA_ERR_NO_DEVICE"])
+
+
+def fwd_host(lib, B=1, Hq=2, Hkv=1, Nq=8, Nk=8, D=128, scale=0.1, causal=0, qh=FAKE, kh=FAKE,
+             vh=FAKE, oh=FAKE, lh=FAKE, q=FAKE, k=FAKE, v=FAKE, o=FAKE, l=FAKE):
+    return lib.fa_fwd_host(qh, kh, vh, oh, lh, q, k, v, o, l, B, Hq, Hkv, Nq, Nk, D, scale, causal,
+                           None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=-1), "FA_ERR_INVALID_ARG"),
+    (dict(D=96), "FA_ERR_UNSUPPORTED"),
+    (dict(Hq=3, Hkv=2), "FA_ERR_INVALID_ARG"),
+    (dict(qh=None), "FA_ERR_INVALID_ARG"),
+    (dict(vh=None), "FA_ERR_INVALID_ARG"),
+    (dict(oh=None), "FA_ERR_INVALID_ARG"),
+    (dict(lh=None), "FA_ERR_INVALID_ARG"),     # lse_host and lse_dev: both or neither
+    (dict(q=FAKE + 4), "FA_ERR_INVALID_ARG"),
+])
+def test_fwd_host_rejects_bad_arguments_on_the_host(lib, kw, code):
+    assert fwd_host(lib, **kw) == E[code]
+
+
+def test_fwd_host_empty_problem_is_a_noop(lib):
+    assert fwd_host(lib, B=0) == 0
+    assert fwd_host(lib, Nq=0) == 0
