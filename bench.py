@@ -312,7 +312,7 @@ def pending_rows(fa, dev, stream, flush, warmup, steps, peaks, peak_src):
     """Kernels built but not yet verified on a B200 (FP8 forward and its
     quantiser, backward): timed on the headline prefill workload only when
     --pending is given, never in a default run."""
-    from exact_tiled_attention_40_b200.inputs import FP8_CASES, hadamard_signs
+    from exact_tiled_attention_40_b200.inputs import FP8_CASES, hadamard_signs, make_dout
     out = {}
     sp = stream.cuda_stream
 
@@ -366,7 +366,7 @@ def pending_rows(fa, dev, stream, flush, warmup, steps, peaks, peak_src):
                                            "unit": "TFLOP/s", "frac": tf / pk,
                                            "peak_source": f"{peak_src} burst bf16 x 2 "
                                                           "(nominal fp8 / bf16 ratio)"}}
-        do = torch.randn(q.shape, generator=gen).to(torch.bfloat16).to(dev)
+        do = make_dout(c, gen).to(dev)
         ob, lb = fa.attention(q, k, v, c.softmax_scale, c.causal)
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
         delta = torch.empty((c.B, c.Hq, c.Nq), dtype=torch.float32, device=dev)

@@ -24,6 +24,10 @@ key lengths; a permutation of the page pool handed out in sequence order as for
 paged decode; then packed Q [total_q, Hq, D], then the K pool and the V pool
 ``randn(num_pages, 16, Hkv, D)``.
 
+Recipe (backward): the prefill case's inputs, then the output gradient dO drawn
+from the same generator after V as ``randn(B, Hq, Nq, D)`` rounded to bf16 (sampled
+rows, where used, come after dO).
+
 Recipe (FP8 forward): the bf16 inputs of the named prefill case, drawn as
 above; the rotation's D signs from their own generator seeded with the case's
 sign seed, ``rand(D) < 0.5`` giving -1.
@@ -44,7 +48,7 @@ __all__ = ["PrefillCase", "DecodeCase", "VarlenCase", "PREFILL_CASES", "DECODE_C
            "VARLEN_CASES", "PagedPrefillCase", "PAGED_PREFILL_CASES", "make_paged_prefill",
            "make_prefill",
            "make_decode", "make_varlen", "varlen_flops",
-           "sample_rows", "hadamard_signs", "Fp8Case", "FP8_CASES"]
+           "sample_rows", "hadamard_signs", "Fp8Case", "FP8_CASES", "make_dout"]
 
 _DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16}
 
@@ -332,6 +336,12 @@ PAGED_PREFILL_CASES = {
         nk=(1024, 8192, 2048, 4096, 3000, 6000, 5120, 1536, 7000, 2500, 4500, 8000, 1800, 3500,
             6500, 5000)),
 }
+
+
+def make_dout(case: PrefillCase, gen: torch.Generator) -> torch.Tensor:
+    """Output gradient dO [B, Hq, Nq, D] for a backward pass, ``randn`` from ``gen``
+    (the case's generator after V) rounded to bf16."""
+    return torch.randn((case.B, case.Hq, case.Nq, case.D), generator=gen).to(torch.bfloat16)
 
 
 def hadamard_signs(D: int, seed: int) -> torch.Tensor:

@@ -27,8 +27,8 @@ import torch
 
 from . import fa
 from .inputs import (DECODE_CASES, FP8_CASES, PAGED_PREFILL_CASES, PREFILL_CASES, VARLEN_CASES,
-                     hadamard_signs, make_decode, make_paged_prefill, make_prefill, make_varlen,
-                     varlen_flops)
+                     hadamard_signs, make_decode, make_dout, make_paged_prefill, make_prefill,
+                     make_varlen, varlen_flops)
 
 
 def main():
@@ -45,7 +45,7 @@ def main():
     if args.op == "bwd":
         c = PREFILL_CASES[args.case]
         q, k, v, gen = make_prefill(c)
-        do = torch.randn((c.B, c.Hq, c.Nq, c.D), generator=gen).to(torch.bfloat16)
+        do = make_dout(c, gen)
         q, k, v, do = q.to(dev), k.to(dev), v.to(dev), do.to(dev)
         o, lse = fa.attention(q, k, v, c.softmax_scale, c.causal)
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)

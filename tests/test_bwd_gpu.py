@@ -24,7 +24,8 @@ import torch
 
 import oracle
 from exact_tiled_attention_40_b200 import fa
-from exact_tiled_attention_40_b200.inputs import PREFILL_CASES, PrefillCase, make_prefill, sample_rows
+from exact_tiled_attention_40_b200.inputs import (PREFILL_CASES, PrefillCase, make_dout,
+                                                  make_prefill, sample_rows)
 
 pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not os.environ.get("FA_PENDING_GPU_TESTS"),
@@ -35,10 +36,6 @@ U = 2.0 ** -7 + 1e-4
 
 def f64(t):
     return t.float().double().numpy()
-
-
-def draw_dout(case, gen):
-    return torch.randn((case.B, case.Hq, case.Nq, case.D), generator=gen).to(torch.bfloat16)
 
 
 def bounds(q, k, v, o, lse, do, scale, causal):
@@ -66,7 +63,7 @@ def bounds(q, k, v, o, lse, do, scale, causal):
 
 def run_case(case):
     q, k, v, gen = make_prefill(case)
-    do = draw_dout(case, gen)
+    do = make_dout(case, gen)
     O, L = oracle.attention(f64(q), f64(k), f64(v), case.softmax_scale, case.causal)
     o = torch.from_numpy(O).to(torch.bfloat16)
     lse = torch.from_numpy(L).to(torch.float32)
@@ -125,7 +122,7 @@ def test_full_size_sampled_dq_rows_and_the_dv_sum(cuda_device):
     sum_j dV_j = sum over the group's heads and queries of dO_i."""
     case = PREFILL_CASES["gqa_b1_hq32_hkv8_n8192_d128_causal"]
     q, k, v, gen = make_prefill(case)
-    do = draw_dout(case, gen)
+    do = make_dout(case, gen)
     rows = sample_rows(case, gen, 2)
     dev = torch.device("cuda", 0)
     qg, kg, vg, dog = q.to(dev), k.to(dev), v.to(dev), do.to(dev)
