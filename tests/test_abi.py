@@ -108,7 +108,17 @@ def test_varlen_empty_batch_is_a_noop(lib):
     assert varlen(lib, B=0) == 0
     assert varlen(lib, tq=0) == 0
     assert varlen(lib, max_q=0) == 0
-    assert varlen(lib, tk=0, k=None, v=None, q=FAKE) in (0, E["FA_ERR_NO_DEVICE"])
+
+
+# The next three calls pass validation, so on a machine with a GPU they would launch
+# kernels on the fake addresses: they run only where no device exists.
+NO_DEVICE_ONLY = pytest.mark.skipif(torch.cuda.is_available(),
+                                    reason="fake pointers must never reach a device")
+
+
+@NO_DEVICE_ONLY
+def test_varlen_without_keys_passes_validation(lib):
+    assert varlen(lib, tk=0, k=None, v=None, q=FAKE) == E["FA_ERR_NO_DEVICE"]
 
 
 def paged(lib, B=2, Hq=4, Hkv=2, max_q=9, maxp=4, npages=10, tq=12, D=128, page=16, scale=0.1,
@@ -160,10 +170,14 @@ def test_quantize_rejects_bad_arguments_on_the_host(lib, kw, code):
     assert lib.fa_last_error_string()
 
 
-def test_quantize_empty_slices_need_no_data_pointers(lib):
+def test_quantize_of_no_slices_is_a_noop(lib):
     assert quant(lib, Z=0) == 0
+
+
+@NO_DEVICE_ONLY
+def test_quantize_empty_slices_need_no_data_pointers(lib):
     # N == 0 still writes scales (1 per slice for group 0), so it reaches the device
-    assert quant(lib, N=0, x=None, codes=None) in (0, E["FA_ERR_NO_DEVICE"])
+    assert quant(lib, N=0, x=None, codes=None, group=0) == E["FA_ERR_NO_DEVICE"]
 
 
 def fp8(lib, B=1, Hq=2, Hkv=1, Nq=8, Nk=8, D=128, scale=0.1, causal=0, q=FAKE, k=FAKE,
@@ -246,9 +260,13 @@ def test_bwd_rejects_bad_arguments_on_the_host(lib, kw, code):
 def test_bwd_empty_problems(lib):
     assert bwd(lib, B=0) == 0
     assert bwd(lib, Nq=0, Nk=0) == 0
-    # no queries but keys: dK = dV = 0 must still be written, so the call reaches the device
-    assert bwd(lib, Nq=0, q=None, o=None, lse=None, do=None, dq=None, delta=None) in (
-        0, E["FA_ERR_NO_DEVICE"])
+
+
+@NO_DEVICE_ONLY
+def test_bwd_without_queries_still_reaches_the_device(lib):
+    # no queries but keys: dK = dV = 0 must still be written
+    assert bwd(lib, Nq=0, q=None, o=None, lse=None, do=None, dq=None,
+               delta=None) == E["FA_ERR_NO_DEVICE"]
 
 
 def fwd_host(lib, B=1, Hq=2, Hkv=1, Nq=8, Nk=8, D=128, scale=0.1, causal=0, qh=FAKE, kh=FAKE,
