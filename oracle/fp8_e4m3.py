@@ -173,14 +173,19 @@ def quantize_rows_f32(x, group_rows: int):
     """E4M3 codes and fp32 scales of x [..., N, D] with the decisions in fp32.
 
     group_rows > 0: one scale per `group_rows` rows (the last group may be
-    short); 0: one scale per [N, D] slice.  Per group: amax = max |x| (fp32),
+    short); 0: one scale per [N, D] slice (1 for an empty slice).  Per group: amax = max |x| (fp32),
     r = fp32(448 / amax), scale = fp32(amax / 448) (both 1 when amax = 0), and
     code = E4M3(fp32(x * r)).  Returns (codes as float64 E4M3 values, scales as
     float32 [..., groups])."""
     x32 = np.asarray(x, dtype=np.float32)
     n = x32.shape[-2]
+    if group_rows == 0:                      # one group per slice, an empty one has scale 1
+        codes = np.zeros(x32.shape, dtype=np.float64)
+        scales = np.ones(x32.shape[:-2] + (1,), dtype=np.float32)
+        if n == 0:
+            return codes, scales
     g = n if group_rows == 0 else group_rows
-    ng = max(1, (n + g - 1) // g) if n else 0
+    ng = (n + g - 1) // g
     codes = np.empty(x32.shape, dtype=np.float64)
     scales = np.empty(x32.shape[:-2] + (ng,), dtype=np.float32)
     for i in range(ng):

@@ -132,6 +132,11 @@ def test_fp32_quantiser_closed_forms():
     c, s = f8.quantize_rows_f32(z, 128)
     np.testing.assert_array_equal(s, np.ones((1, 2), np.float32))   # zero group: scale 1
     assert np.all(c == 0)
+    # an empty slice: no codes, scale 1 (one group per slice)
+    c, s = f8.quantize_rows_f32(np.zeros((2, 0, 8), np.float32), 0)
+    assert c.shape == (2, 0, 8) and s.shape == (2, 1) and np.all(s == 1)
+    c, s = f8.quantize_rows_f32(np.zeros((2, 0, 8), np.float32), 128)
+    assert s.shape == (2, 0)
     # a value far below the group's amax rounds to zero with its sign kept
     t = np.array([[[448.0, -1e-6]]], np.float32)
     c, _ = f8.quantize_rows_f32(t, 128)
