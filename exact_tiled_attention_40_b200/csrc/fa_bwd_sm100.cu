@@ -190,10 +190,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // work: key tile j of (b, hkv)
-  const int n_kt = (p.Nk + kBM - 1) / kBM;
-  const int j = blockIdx.x % n_kt;
-  const int bh_kv = blockIdx.x / n_kt;
+  // work: key tile j of (b, hkv); CTAs in order of j, so under the causal mask the
+  // heaviest tiles (seen by the most query tiles) start first
+  const int nkvh = p.B * p.Hkv;
+  const int j = blockIdx.x / nkvh;
+  const int bh_kv = blockIdx.x - j * nkvh;
   const int b = bh_kv / p.Hkv;
   const int hkv = bh_kv - b * p.Hkv;
   const int G = p.Hq / p.Hkv;
@@ -407,9 +408,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
+  // work: query tile i of (b, h); CTAs from the last query tile down, so under the
+  // causal mask the heaviest tiles (the most key tiles) start first
   const int n_qt = (p.Nq + kBM - 1) / kBM;
-  const int i = blockIdx.x % n_qt;
-  const int bh = blockIdx.x / n_qt;                  // b * Hq + h
+  const int nbh = p.B * p.Hq;
+  const int i = n_qt - 1 - static_cast<int>(blockIdx.x) / nbh;
+  const int bh = static_cast<int>(blockIdx.x) - (n_qt - 1 - i) * nbh;   // b * Hq + h
   const int b = bh / p.Hq;
   const int h = bh - b * p.Hq;
   const int hkv = h / (p.Hq / p.Hkv);
