@@ -493,6 +493,17 @@ int fa_decode_paged_noalloc(const void* q, const void* kcache, const void* vcach
                                reinterpret_cast<cudaStream_t>(stream), dev);
 }
 
+int fa_selftest_wait_timeout(unsigned int limit_us, int* gave_up, fa_stream_t stream) {
+  using namespace fa;
+  if (limit_us == 0 || limit_us > 1000000u)
+    return set_error(FA_ERR_INVALID_ARG, "limit_us must be in [1, 1000000] (got %u)", limit_us);
+  if (gave_up && (reinterpret_cast<uintptr_t>(gave_up) & 3u))
+    return set_error(FA_ERR_INVALID_ARG, "gave_up must be 4-byte aligned");
+  int dev, rc;
+  if ((rc = current_sm100(&dev)) != FA_OK) return rc;
+  return launch_wait_selftest(limit_us, gave_up, reinterpret_cast<cudaStream_t>(stream), dev);
+}
+
 const char* fa_last_error_string(void) { return fa::g_msg; }
 
 int fa_device_status(void) {

@@ -91,6 +91,9 @@ int launch_fwd_host(const void* q_host, const void* k_host, const void* v_host, 
                     int causal, cudaStream_t stream, int device);
 void release_host_pipeline_resources();
 
+// One bounded wait that nothing satisfies, given up after limit_us (validated).
+int launch_wait_selftest(unsigned limit_us, int* gave_up, cudaStream_t stream, int device);
+
 // Release cached per-device resources owned by the decode path.
 void release_decode_resources();
 

@@ -44,6 +44,7 @@ _SIGS = {
     "fa_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _I, _I, _P]),
     "fa_decode_paged_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _I, _I,
                                      _P]),
+    "fa_selftest_wait_timeout": (_I, [ctypes.c_uint, _P, _P]),
     "fa_last_error_string": (ctypes.c_char_p, []),
     "fa_device_status": (_I, []),
     "fa_release": (None, []),
@@ -394,6 +395,17 @@ def decode_paged_noalloc(q, kcache, vcache, block_table, seq_lens, o, lse=None, 
 def device_status() -> int:
     """Synchronise and read/clear the device error word (FA_* code)."""
     return lib().fa_device_status()
+
+
+def selftest_wait_timeout(limit_us: int = 20000, device=None):
+    """Run the bounded-wait self-test (a wait nothing satisfies, given up after
+    limit_us) and return (fa_device_status() code, whether the wait gave up)."""
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    flag = torch.full((1,), -1, dtype=torch.int32, device=device)
+    _check(lib().fa_selftest_wait_timeout(int(limit_us), _ptr(flag), _stream(device)),
+           "fa_selftest_wait_timeout")
+    status = device_status()
+    return status, int(flag.item()) == 1
 
 
 def last_error() -> str:

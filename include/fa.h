@@ -224,6 +224,18 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
            int Nq, int Nk, int D, float scale, int causal, fa_stream_t stream);
 
 /*
+ * Self-test of the bounded in-kernel waits (failure detection without a fault).
+ * Launches one thread that waits on a barrier nothing ever completes; after
+ * limit_us microseconds (1 .. 1000000) the wait gives up, sets the timeout bit
+ * of the device error word and the kernel returns.  The next fa_device_status()
+ * then reports FA_ERR_DEVICE_TIMEOUT (and clears the word); the context stays
+ * usable.  gave_up (device int, may be NULL) receives 1 if the wait gave up,
+ * 0 if it was satisfied.  Every other kernel of the library waits through the
+ * same routine, with a limit of 2 s.
+ */
+int fa_selftest_wait_timeout(unsigned int limit_us, int* gave_up, fa_stream_t stream);
+
+/*
  * Merge of partial attention results over disjoint key sets (the combine step
  * of the split-KV decode, exposed for sequence-sharded prefill: each rank's
  * queries meet the K/V chunks of every rank and fold each chunk's result in).

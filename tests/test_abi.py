@@ -292,3 +292,13 @@ def test_fwd_host_rejects_bad_arguments_on_the_host(lib, kw, code):
 def test_fwd_host_empty_problem_is_a_noop(lib):
     assert fwd_host(lib, B=0) == 0
     assert fwd_host(lib, Nq=0) == 0
+
+
+@pytest.mark.parametrize("limit,ptr", [(0, None), (2_000_000, None), (100, FAKE + 2)])
+def test_wait_selftest_rejects_bad_arguments(lib, limit, ptr):
+    assert lib.fa_selftest_wait_timeout(limit, ptr, None) == E["FA_ERR_INVALID_ARG"]
+
+
+@NO_DEVICE_ONLY
+def test_wait_selftest_needs_a_device(lib):
+    assert lib.fa_selftest_wait_timeout(100, None, None) == E["FA_ERR_NO_DEVICE"]
