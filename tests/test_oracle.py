@@ -443,3 +443,24 @@ def test_pins_catch_a_missing_delta_term():
                                                          torch.from_numpy(v), scale=0.5)
     o.backward(torch.from_numpy(do))
     assert np.max(np.abs(dq_bad - tq.grad.numpy())) > 1e-3
+
+
+def test_backward_closed_forms():
+    """One key: P = 1, so dV sums dO over the group's query heads and rows, and dS =
+    dO.v - dO.o = 0 gives dQ = dK = 0.  Zero queries (uniform weights 1/Nk, no
+    mask): dV_j = sum_i dO_i / Nk for every key j."""
+    q, k, v = rand((1, 4, 3, 8), 150), rand((1, 2, 1, 8), 151), rand((1, 2, 1, 8), 152)
+    do = rand((1, 4, 3, 8), 153)
+    O, L = oracle.attention(q, k, v, 0.3, False)
+    dq, dk, dv = oracle.attention_backward(q, k, v, O, L, do, 0.3, False)
+    np.testing.assert_allclose(dq, 0, atol=1e-12)
+    np.testing.assert_allclose(dk, 0, atol=1e-12)
+    want = do.reshape(1, 2, 2, 3, 8).sum(axis=(2, 3))[:, :, None, :]
+    np.testing.assert_allclose(dv, want, atol=1e-12)
+    qz = np.zeros((1, 2, 5, 8))
+    k2, v2 = rand((1, 2, 6, 8), 154), rand((1, 2, 6, 8), 155)
+    do2 = rand((1, 2, 5, 8), 156)
+    O2, L2 = oracle.attention(qz, k2, v2, 0.3, False)
+    _, _, dv2 = oracle.attention_backward(qz, k2, v2, O2, L2, do2, 0.3, False)
+    np.testing.assert_allclose(dv2, np.repeat(do2.sum(axis=2, keepdims=True) / 6, 6, axis=2),
+                               atol=1e-12)
