@@ -12,11 +12,7 @@ P costs < 1e-4 relative.  So for every element
     |d dK_jd| <= (2^-7 + 1e-4) scale sum_i |dS_ij| |Q_id|,
     |d dQ_id| <= (2^-7 + 1e-4) scale sum_j |dS_ij| |K_jd|,
 plus 1e-6 (summed over the query heads of a KV head for dK, dV).
-
-These tests wait for their first run on a B200: they run when the environment
-variable FA_PENDING_GPU_TESTS is set.
 """
-import os
 
 import numpy as np
 import pytest
@@ -27,9 +23,7 @@ from exact_tiled_attention_40_b200 import fa
 from exact_tiled_attention_40_b200.inputs import (PREFILL_CASES, PrefillCase, make_dout,
                                                   make_prefill, sample_rows)
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(not os.environ.get("FA_PENDING_GPU_TESTS"),
-                                 reason="awaiting a first B200 run: FA_PENDING_GPU_TESTS")]
+pytestmark = pytest.mark.gpu
 
 U = 2.0 ** -7 + 1e-4
 

@@ -3,11 +3,7 @@ sits in the middle of a larger allocation whose margins hold a canary pattern
 (NaN for inputs, so a stray read shows up in the results; a fixed bit pattern
 for outputs, so a stray write shows up in the margins).  After the call the
 margins must be untouched and the results must still match the oracle.
-
-These tests wait for their first run on a B200: they run when the environment
-variable FA_PENDING_GPU_TESTS is set.
 """
-import os
 
 import numpy as np
 import pytest
@@ -19,9 +15,7 @@ from exact_tiled_attention_40_b200.inputs import (DecodeCase, PrefillCase, Varle
                                                   make_decode, make_dout, make_prefill,
                                                   make_varlen)
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(not os.environ.get("FA_PENDING_GPU_TESTS"),
-                                 reason="awaiting a first B200 run: FA_PENDING_GPU_TESTS")]
+pytestmark = pytest.mark.gpu
 
 PAD_BYTES = 8192          # margin on each side (a multiple of 16: alignment is kept)
 

@@ -3,11 +3,7 @@ satisfies gives up after its limit, the host reads FA_ERR_DEVICE_TIMEOUT from
 fa_device_status(), and the context stays usable (a forward right after it
 still matches the oracle).  Out-of-range indices read from device memory are
 covered by tests/test_decode_gpu.py and tests/test_varlen_gpu.py.
-
-This test waits for its first run on a B200: it runs when the environment
-variable FA_PENDING_GPU_TESTS is set.
 """
-import os
 
 import numpy as np
 import pytest
@@ -17,9 +13,7 @@ import oracle
 from exact_tiled_attention_40_b200 import fa
 from exact_tiled_attention_40_b200.inputs import PrefillCase, make_prefill
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(not os.environ.get("FA_PENDING_GPU_TESTS"),
-                                 reason="awaiting a first B200 run: FA_PENDING_GPU_TESTS")]
+pytestmark = pytest.mark.gpu
 
 
 def test_a_wait_that_runs_out_is_reported_and_the_context_survives(cuda_device):

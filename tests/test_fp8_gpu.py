@@ -20,11 +20,7 @@ P to E4M3 before P V; the tolerances derive from it:
   * LSE is computed from the unrounded p: |dLSE| <= 2e-4 + 2^-13 S_abs, with
     S_abs = max_j scale * sum_d |q_d k_jd|, allowing the tensor core's fp32
     accumulation of the E4M3 products a relative error of 2^-13.
-
-These tests wait for their first run on a B200: they run when the environment
-variable FA_PENDING_GPU_TESTS is set.
 """
-import os
 
 import numpy as np
 import pytest
@@ -36,9 +32,7 @@ from exact_tiled_attention_40_b200 import fa
 from exact_tiled_attention_40_b200.inputs import (FP8_CASES, PrefillCase, hadamard_signs,
                                                   make_prefill, sample_rows)
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(not os.environ.get("FA_PENDING_GPU_TESTS"),
-                                 reason="awaiting a first B200 run: FA_PENDING_GPU_TESTS")]
+pytestmark = pytest.mark.gpu
 
 
 def f32(t):

@@ -3,11 +3,7 @@ forward chunk by chunk) gives exactly fa_fwd's result: the same kernel runs on
 each chunk's slice, so O and LSE must match bit for bit; the shapes cover the
 chunk plans (groups of one sequence, several sequences per chunk, a ragged
 last chunk, no keys).
-
-These tests wait for their first run on a B200: they run when the environment
-variable FA_PENDING_GPU_TESTS is set.
 """
-import os
 
 import pytest
 import torch
@@ -15,9 +11,7 @@ import torch
 from exact_tiled_attention_40_b200 import fa
 from exact_tiled_attention_40_b200.inputs import PrefillCase, make_prefill
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(not os.environ.get("FA_PENDING_GPU_TESTS"),
-                                 reason="awaiting a first B200 run: FA_PENDING_GPU_TESTS")]
+pytestmark = pytest.mark.gpu
 
 CASES = [
     PrefillCase("host_groups", 1, 32, 8, 1024, 1024, 128, seed=100, causal=True),

@@ -6,11 +6,7 @@ as one rank (no exchange) and as four ranks one after another on the same
 device with their K/V chunks handed in per step (no rank waits for another),
 and compared with the fp64 oracle on the whole sequence within the forward's
 tolerances (max |dO| <= 2e-2, max |dLSE| <= 1e-3).
-
-These tests wait for their first run on a B200: they run when the environment
-variable FA_PENDING_GPU_TESTS is set.
 """
-import os
 
 import numpy as np
 import pytest
@@ -20,9 +16,7 @@ import oracle
 from exact_tiled_attention_40_b200 import fa, ring
 from exact_tiled_attention_40_b200.inputs import PrefillCase, make_prefill
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(not os.environ.get("FA_PENDING_GPU_TESTS"),
-                                 reason="awaiting a first B200 run: FA_PENDING_GPU_TESTS")]
+pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("D", [64, 128])
