@@ -1,6 +1,7 @@
 // C-ABI entry points: argument validation on the host, error reporting and the
 // per-device error word.  Every compute step runs in the kernels of
 // fa_fwd_sm100.cu and fa_decode_sm100.cu; there is no host fallback.
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdint>
@@ -19,7 +20,11 @@ thread_local char g_msg[512] = "";
 __device__ int g_error_word;   // see kErrTimeout / kErrBadIndex
 std::mutex g_err_mu;
 int* g_err_ptr[64] = {};
+int g_err_gen[64] = {};
+std::atomic<int> g_cache_gen{1};
 }  // namespace
+
+int cache_generation() { return g_cache_gen.load(std::memory_order_acquire); }
 
 int set_error(int code, const char* fmt, ...) {
   va_list ap;
@@ -32,10 +37,12 @@ int set_error(int code, const char* fmt, ...) {
 int* device_error_word(int device) {
   if (device < 0 || device >= 64) return nullptr;
   std::lock_guard<std::mutex> g(g_err_mu);
-  if (!g_err_ptr[device]) {
+  const int gen = cache_generation();
+  if (!g_err_ptr[device] || g_err_gen[device] != gen) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
     g_err_ptr[device] = static_cast<int*>(p);
+    g_err_gen[device] = gen;
   }
   return g_err_ptr[device];
 }
@@ -485,8 +492,9 @@ int fa_decode_paged_noalloc(const void* q, const void* kcache, const void* vcach
   if (static_cast<long long>(max_pages_per_seq) * 16 > 0x7fffffffLL)
     return set_error(FA_ERR_INVALID_ARG, "max_pages_per_seq too large");
   int dev, rc;
-  // The scratch bound is checked before the device is touched.
-  if ((rc = check_decode_noalloc(B, Hq, Hkv, max_pages_per_seq)) != FA_OK) return rc;
+  // Problems that no schedule fits are rejected before the device is touched;
+  // the plan for the device's SM count is checked again at launch.
+  if ((rc = check_decode_noalloc(B, Hq, Hkv, max_pages_per_seq, 0)) != FA_OK) return rc;
   if ((rc = current_sm100(&dev)) != FA_OK) return rc;
   return launch_decode_noalloc(q, kcache, vcache, block_table, seq_lens, o, lse, B, Hq, Hkv,
                                max_pages_per_seq, num_pages, scale,
@@ -521,6 +529,9 @@ int fa_device_status(void) {
   cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int));
   if (word & kErrTimeout)
     return set_error(FA_ERR_DEVICE_TIMEOUT, "a bounded in-kernel wait ran out (word 0x%x)", word);
+  if (word & kErrDiverged)
+    return set_error(FA_ERR_DEVICE_DIVERGED,
+                     "a tensor-memory access found its warp diverged (word 0x%x)", word);
   return set_error(FA_ERR_DEVICE_INDEX, "out-of-range block-table entry or length (word 0x%x)",
                    word);
 }
@@ -528,6 +539,8 @@ int fa_device_status(void) {
 void fa_release(void) {
   fa::release_decode_resources();
   fa::release_host_pipeline_resources();
+  // cached device addresses and kernel attributes are looked up again on next use
+  fa::g_cache_gen.fetch_add(1, std::memory_order_acq_rel);
 }
 
 int fa_version(void) { return 100; }

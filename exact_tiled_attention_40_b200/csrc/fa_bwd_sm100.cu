@@ -141,12 +141,13 @@ __device__ __forceinline__ void mma_tmem_x_tile(uint32_t d, uint32_t a, uint64_t
 
 // Store a row of D fp32 TMEM values (columns t0 ..), times `mul`, as bf16.
 template <int D>
-__device__ __forceinline__ void store_row_bf16(uint32_t t0, float mul, uint16_t* dst, bool valid) {
+__device__ __forceinline__ void store_row_bf16(uint32_t t0, float mul, uint16_t* dst, bool valid,
+                                               int* err) {
 #pragma unroll 1
   for (int c = 0; c < D / 32; ++c) {
     uint32_t v[32];
-    tmem_ld32(t0 + 32 * c, v);
-    tmem_wait_ld();
+    tmem_ld32(t0 + 32 * c, v, err);
+    tmem_wait_ld(err);
     uint32_t pk[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e)
@@ -333,9 +334,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t sv[32], dv[32];
-        tmem_ld32(tS + 32 * c, sv);
-        tmem_ld32(tP + 32 * c, dv);
-        tmem_wait_ld();
+        tmem_ld32(tS + 32 * c, sv, p.err);
+        tmem_ld32(tP + 32 * c, dv, p.err);
+        tmem_wait_ld(p.err);
         const int q0 = i * kBM + 32 * c;
         uint32_t pk[16], dk[16];
 #pragma unroll
@@ -358,10 +359,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           dk[e >> 1] = pack_bf16x2(de[0], de[1]);
         }
         // the packed pairs go over columns already read (16 c .. 16 c + 15)
-        tmem_st16(tS + 16 * c, pk);
-        tmem_st16(tP + 16 * c, dk);
+        tmem_st16(tS + 16 * c, pk, p.err);
+        tmem_st16(tP + 16 * c, dk, p.err);
       }
-      tmem_wait_st();
+      tmem_wait_st(p.err);
       tc_fence_before();
       mbar_arrive(p_full);
     }
@@ -377,8 +378,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           store_zero_row<D>(p.dk + orow);
         }
       } else {
-        store_row_bf16<D>(tmem + lane_base + 256, 1.f, p.dv + orow, valid);
-        store_row_bf16<D>(tmem + lane_base + 256 + D, p.scale, p.dk + orow, valid);
+        store_row_bf16<D>(tmem + lane_base + 256, 1.f, p.dv + orow, valid, p.err);
+        store_row_bf16<D>(tmem + lane_base + 256 + D, p.scale, p.dk + orow, valid, p.err);
       }
     }
   }
@@ -549,9 +550,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t sv[32], dv[32];
-        tmem_ld32(tS + 32 * c, sv);
-        tmem_ld32(tP + 32 * c, dv);
-        tmem_wait_ld();
+        tmem_ld32(tS + 32 * c, sv, p.err);
+        tmem_ld32(tP + 32 * c, dv, p.err);
+        tmem_wait_ld(p.err);
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
@@ -566,9 +567,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[e >> 1] = pack_bf16x2(p0 * (__uint_as_float(dv[e]) - dl),
                                    p1 * (__uint_as_float(dv[e + 1]) - dl));
         }
-        tmem_st16(tS + 16 * c, pk);     // over columns already read
+        tmem_st16(tS + 16 * c, pk, p.err);     // over columns already read
       }
-      tmem_wait_st();
+      tmem_wait_st(p.err);
       tc_fence_before();
       mbar_arrive(ds_full);
     }
@@ -579,7 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (n_kt == 0) {
         if (row < p.Nq) store_zero_row<D>(dst);
       } else {
-        store_row_bf16<D>(tmem + lane_base + 256, p.scale, dst, row < p.Nq);
+        store_row_bf16<D>(tmem + lane_base + 256, p.scale, dst, row < p.Nq, p.err);
       }
     }
   }
@@ -609,12 +610,12 @@ int launch_bwd_typed(const void* q, const void* k, const void* v, const void* o,
                      float* delta, int B, int Hq, int Hkv, int Nq, int Nk, float scale,
                      int causal, cudaStream_t stream, int device) {
   using L = BwdLayout<D>;
-  static bool attr_done[64] = {};
+  static int attr_gen[64] = {};
   static std::mutex mu;
   {
     std::lock_guard<std::mutex> g(mu);
     if (device < 0 || device >= 64) return set_error(FA_ERR_CUDA, "device ordinal out of range");
-    if (!attr_done[device]) {
+    if (attr_gen[device] != cache_generation()) {
       cudaError_t e = cudaFuncSetAttribute(fa_bwd_dkdv_kernel<D>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            L::kSmemBytes);
@@ -623,7 +624,7 @@ int launch_bwd_typed(const void* q, const void* k, const void* v, const void* o,
                                  L::kSmemBytes);
       if (e != cudaSuccess)
         return set_error(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-      attr_done[device] = true;
+      attr_gen[device] = cache_generation();
     }
   }
   BwdParams prm;

@@ -900,17 +900,17 @@ int launch_kernels(const DecodeParams& prm, const DecodePlan& pl, const CUtensor
                      (prm.hb_in_smem ? (prm.B + 1) * 4 : 0);
     {
       // the shared-memory limit is a property of the function on each device
-      static bool attr_done[64] = {};
+      static int attr_gen[64] = {};
       static std::mutex mu;
       std::lock_guard<std::mutex> g(mu);
       if (device < 0 || device >= 64) return set_error(FA_ERR_CUDA, "device ordinal out of range");
-      if (!attr_done[device]) {
+      if (attr_gen[device] != cache_generation()) {
         cudaError_t e = cudaFuncSetAttribute(fa_decode_stream_kernel<G>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kStreamSmemBudget + 1024 + kHbSmemMax * 4);
         if (e != cudaSuccess)
           return set_error(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-        attr_done[device] = true;
+        attr_gen[device] = cache_generation();
       }
     }
     // The stream and merge kernels are launched with programmatic serialization:
@@ -1065,31 +1065,53 @@ static __device__ __align__(256) float g_decode_scratch[kNoAllocScratchBytes / s
 namespace {
 std::mutex g_scratch_mu;
 float* g_scratch_ptr[64] = {};
+int g_scratch_gen[64] = {};
 
 // Device address of g_decode_scratch on `device` (which must be current).  In
 // host code the array's name is only a host-side stand-in; the address a kernel
-// may use comes from cudaGetSymbolAddress, looked up once per device.
+// may use comes from cudaGetSymbolAddress, looked up once per device (and again
+// after fa_release(), which a caller makes after resetting the device).
 int scratch_address(int device, float** out) {
   if (device < 0 || device >= 64) return set_error(FA_ERR_CUDA, "device ordinal out of range");
   std::lock_guard<std::mutex> g(g_scratch_mu);
-  if (!g_scratch_ptr[device]) {
+  const int gen = cache_generation();
+  if (!g_scratch_ptr[device] || g_scratch_gen[device] != gen) {
     void* p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess || p == nullptr)
       return set_error(FA_ERR_CUDA, "cudaGetSymbolAddress(decode scratch): %s",
                        cudaGetErrorString(e));
     g_scratch_ptr[device] = static_cast<float*>(p);
+    g_scratch_gen[device] = gen;
   }
   *out = g_scratch_ptr[device];
   return FA_OK;
 }
 
-// Plan that fits the fixed scratch: the streamed schedule as is when it fits;
-// the direct schedule with chunks widened until its partials fit.
+// Direct schedule with its page chunks widened until the partials fit.
+DecodePlan widen_direct(int B, int Hq, int Hkv, int max_pages_per_seq) {
+  DecodePlan pl;
+  pl.streamed = false;
+  pl.pps = direct_pps(B, max_pages_per_seq);
+  pl.nsplit = (max_pages_per_seq + pl.pps - 1) / pl.pps;
+  finish_plan(pl, B, Hq, Hkv);
+  while (pl.bytes > kNoAllocScratchBytes && pl.nsplit > 1) {
+    pl.pps *= 2;
+    pl.nsplit = (max_pages_per_seq + pl.pps - 1) / pl.pps;
+    finish_plan(pl, B, Hq, Hkv);
+  }
+  return pl;
+}
+
+// Plan that fits the fixed scratch on a device with `nsm` SMs (0: no device
+// known, which plans the direct schedule, the one with the smallest need).
+// The streamed schedule (Hkv <= 8) is kept when it fits, if need be with fewer
+// dynamic units (each then covers more half-pages) or none; otherwise the
+// direct schedule with widened chunks, which needs only B * Hq rows at one
+// chunk per sequence.
 int plan_noalloc(int B, int Hq, int Hkv, int max_pages_per_seq, int nsm, DecodePlan* out) {
   DecodePlan pl = make_plan(B, Hq, Hkv, max_pages_per_seq, nsm);
   if (pl.streamed && pl.bytes > kNoAllocScratchBytes) {
-    // fewer dynamic units (each then covers more half-pages), or none
     const long long rows_fit =
         (static_cast<long long>(kNoAllocScratchBytes) - (static_cast<long long>(B) + 2) * 4) /
         ((kDecD + 1) * 4) / Hq;
@@ -1097,29 +1119,21 @@ int plan_noalloc(int B, int Hq, int Hkv, int max_pages_per_seq, int nsm, DecodeP
     pl.dyn_units_cap = cap > 0 ? static_cast<int>(std::min<long long>(cap, pl.dyn_units_cap)) : 0;
     finish_plan(pl, B, Hq, Hkv);
   }
-  if (!pl.streamed) {
-    while (pl.bytes > kNoAllocScratchBytes && pl.nsplit > 1) {
-      pl.pps *= 2;
-      pl.nsplit = (max_pages_per_seq + pl.pps - 1) / pl.pps;
-      finish_plan(pl, B, Hq, Hkv);
-    }
-  }
+  if (pl.bytes > kNoAllocScratchBytes) pl = widen_direct(B, Hq, Hkv, max_pages_per_seq);
   if (pl.bytes > kNoAllocScratchBytes)
     return set_error(FA_ERR_INVALID_ARG,
                      "fa_decode_paged_noalloc: this problem needs %zu bytes of scratch; the fixed "
-                     "scratch holds %zu bytes (partial rows: (SMs + B) * Hq for Hkv <= 8, "
-                     "B * Hq for Hkv > 8, each %d bytes)",
-                     pl.bytes, kNoAllocScratchBytes, (kDecD + 1) * 4);
+                     "scratch holds %zu bytes (partial rows of %d bytes: at least B * Hq = %lld)",
+                     pl.bytes, kNoAllocScratchBytes, (kDecD + 1) * 4,
+                     static_cast<long long>(B) * Hq);
   *out = pl;
   return FA_OK;
 }
 }  // namespace
 
-int check_decode_noalloc(int B, int Hq, int Hkv, int max_pages_per_seq) {
-  // Host-side bound check (before the device is touched): the SM count is not
-  // known here, so the streamed schedule is checked against 148 SMs, the B200's.
+int check_decode_noalloc(int B, int Hq, int Hkv, int max_pages_per_seq, int nsm) {
   DecodePlan pl;
-  return plan_noalloc(B, Hq, Hkv, max_pages_per_seq, 148, &pl);
+  return plan_noalloc(B, Hq, Hkv, max_pages_per_seq, nsm, &pl);
 }
 
 int launch_decode_noalloc(const void* q, const void* kcache, const void* vcache,

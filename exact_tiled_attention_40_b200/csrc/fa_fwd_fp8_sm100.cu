@@ -525,11 +525,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         uint32_t s[128];
-        tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
-        tmem_wait_ld();
+        tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]), p.err);
+        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]), p.err);
+        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]), p.err);
+        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]), p.err);
+        tmem_wait_ld(p.err);
         const int kbase = j * kBN;
         const bool need_mask =
             (kbase + kBN > p.Nk) || (p.causal && kbase + kBN - 1 > tile_first + off);
@@ -564,11 +564,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
           for (int cc = 0; cc < kD / 32; ++cc) {
             uint32_t ov[32];
-            tmem_ld32(tO + 32 * cc, ov);
-            tmem_wait_ld();
+            tmem_ld32(tO + 32 * cc, ov, p.err);
+            tmem_wait_ld(p.err);
 #pragma unroll
             for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-            tmem_st32(tO + 32 * cc, ov);
+            tmem_st32(tO + 32 * cc, ov, p.err);
           }
         }
         // the half-precision variant exponentiates x - m_ref (small for the
@@ -606,9 +606,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               pk[e] = pack_e4m3x4(p0, p1, p2, p3);
             }
           }
-          tmem_st8(tS + 8 * cq, pk);
+          tmem_st8(tS + 8 * cq, pk, p.err);
           if (cq == 1) {                           // keys 0-63 of P are in place
-            tmem_wait_st();
+            tmem_wait_st(p.err);
             tc_fence_before();
             mbar_arrive(p_half(t, 0));
           }
@@ -616,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float sa, sb;
         f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), sa, sb);
         l += sa + sb;
-        tmem_wait_st();
+        tmem_wait_st(p.err);
         tc_fence_before();
         mbar_arrive(p_half(t, 1));
       }
@@ -632,8 +632,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int cc = 0; cc < kD / 32; ++cc) {
           uint32_t ov[32];
-          tmem_ld32(tO + 32 * cc, ov);
-          tmem_wait_ld();
+          tmem_ld32(tO + 32 * cc, ov, p.err);
+          tmem_wait_ld(p.err);
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
@@ -694,18 +694,18 @@ int launch_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* 
                    int Hq, int Hkv, int Nq, int Nk, float scale, int causal, cudaStream_t stream,
                    int device) {
   using L = Fp8Layout;
-  static bool attr_done[64] = {};
+  static int attr_gen[64] = {};
   static std::mutex mu;
   {
     std::lock_guard<std::mutex> g(mu);
     if (device < 0 || device >= 64) return set_error(FA_ERR_CUDA, "device ordinal out of range");
-    if (!attr_done[device]) {
+    if (attr_gen[device] != cache_generation()) {
       cudaError_t e = cudaFuncSetAttribute(fa_fwd_fp8_kernel,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            L::kSmemBytes);
       if (e != cudaSuccess)
         return set_error(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-      attr_done[device] = true;
+      attr_gen[device] = cache_generation();
     }
   }
   CUtensorMap tq, tk, tv;

@@ -645,11 +645,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         uint32_t s[128];
-        tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
-        tmem_wait_ld();
+        tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]), p.err);
+        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]), p.err);
+        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]), p.err);
+        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]), p.err);
+        tmem_wait_ld(p.err);
         const int kbase = j * kBN;
         const bool need_mask =
             (kbase + kBN > it.nk) || (p.causal && kbase + kBN - 1 > tile_first + off);
@@ -687,11 +687,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             uint32_t ov[32];
-            tmem_ld32(tO + 32 * c, ov);
-            tmem_wait_ld();
+            tmem_ld32(tO + 32 * c, ov, p.err);
+            tmem_wait_ld(p.err);
 #pragma unroll
             for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-            tmem_st32(tO + 32 * c, ov);
+            tmem_st32(tO + 32 * c, ov, p.err);
           }
         }
         const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
@@ -712,9 +712,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               sum2[e & 3] = f2_add(sum2[e & 3], f2_pack(p0, p1));
               pk[e] = BF16 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
             }
-            tmem_st16(tS + 16 * c, pk);
+            tmem_st16(tS + 16 * c, pk, p.err);
             if (c == 1) {                        // keys 0-63 of P are in place
-              tmem_wait_st();
+              tmem_wait_st(p.err);
               tc_fence_before();
               mbar_arrive(p_half(t, 0));
             }
@@ -739,9 +739,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               sum2[e & 3] = f2_add(sum2[e & 3], f2_pack(p0, p1));
               pk[e] = BF16 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
             }
-            tmem_st16(tS + 16 * c, pk);
+            tmem_st16(tS + 16 * c, pk, p.err);
             if (c == 1) {                        // keys 0-63 of P are in place
-              tmem_wait_st();
+              tmem_wait_st(p.err);
               tc_fence_before();
               mbar_arrive(p_half(t, 0));
             }
@@ -750,7 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float sa, sb;
         f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), sa, sb);
         l += sa + sb;
-        tmem_wait_st();
+        tmem_wait_st(p.err);
         tc_fence_before();
         mbar_arrive(p_half(t, 1));
       }
@@ -765,8 +765,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t ov[32];
-          tmem_ld32(tO + 32 * c, ov);
-          tmem_wait_ld();
+          tmem_ld32(tO + 32 * c, ov, p.err);
+          tmem_wait_ld(p.err);
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -843,12 +843,12 @@ int launch_typed(const void* q, const void* k, const void* v, void* o, float* ls
   const bool paged = la.block_table != nullptr;
   using L = FwdLayout<D, false>;
   using LR = FwdLayout<D, true>;   // ragged and paged batches
-  static bool attr_done[64] = {};
+  static int attr_gen[64] = {};
   static std::mutex mu;
   {
     std::lock_guard<std::mutex> g(mu);
     if (device < 0 || device >= 64) return set_error(FA_ERR_CUDA, "device ordinal out of range");
-    if (!attr_done[device]) {
+    if (attr_gen[device] != cache_generation()) {
       cudaError_t e = cudaFuncSetAttribute(fa_fwd_kernel<D, BF16, kDense>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            L::kSmemBytes);
@@ -860,7 +860,7 @@ int launch_typed(const void* q, const void* k, const void* v, void* o, float* ls
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, LR::kSmemBytes);
       if (e != cudaSuccess)
         return set_error(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-      attr_done[device] = true;
+      attr_gen[device] = cache_generation();
     }
   }
   CUtensorMap tq, tk, tv;

@@ -28,6 +28,12 @@ int encode_tensor_map_u8(CUtensorMap* m, const void* base, int rank, const uint6
 // Number of SMs of `device` (cached per device), 0 if it cannot be read.
 int device_sm_count(int device);
 
+// Generation of the per-device host caches that depend on the device's context
+// (device addresses of the library's __device__ symbols, kernel attributes).
+// Starts at 1; fa_release() moves it on, so every such cache is rebuilt on its
+// next use (needed after cudaDeviceReset, which gives the device a new context).
+int cache_generation();
+
 // Wall-time limit of every bounded wait inside a kernel.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
@@ -101,8 +107,9 @@ void release_decode_resources();
 constexpr size_t kNoAllocScratchBytes = 16u << 20;   // 16 MiB
 
 // Host-side check that a problem fits the fixed scratch of
-// fa_decode_paged_noalloc (no device needed).  Returns an FA_* status.
-int check_decode_noalloc(int B, int Hq, int Hkv, int max_pages_per_seq);
+// fa_decode_paged_noalloc on a device with `nsm` SMs; nsm = 0 checks the
+// smallest need of any schedule, without a device.  Returns an FA_* status.
+int check_decode_noalloc(int B, int Hq, int Hkv, int max_pages_per_seq, int nsm);
 
 // Split-KV paged decode whose partials live in the library's fixed scratch
 // array; allocates nothing.  `device` must be the current device.

@@ -10,8 +10,34 @@ namespace fa {
 
 // Device-side error word, read and cleared by fa_device_status().
 // Bit 0: a bounded wait ran out; bit 1: an index read from device memory
-// (block table entry or sequence length) was out of range.
-enum : int { kErrTimeout = 1, kErrBadIndex = 2 };
+// (block table entry or sequence length) was out of range; bit 2 (debug builds
+// only): a warp-collective tensor-memory instruction found its warp diverged.
+enum : int { kErrTimeout = 1, kErrBadIndex = 2, kErrDiverged = 4 };
+
+// FA_DEBUG=1 builds check, before every tensor-memory load, store and their
+// waits (warp-collective tcgen05 instructions), that all 32 lanes of the warp
+// are converged.
+// Those instructions are .sync.aligned: a warp that reaches one with some lanes
+// on another path waits for lanes that never come, a hang that no bounded
+// mbarrier wait can end.  On a diverged warp the check sets kErrDiverged in the
+// error word and skips the instruction (its result is then garbage, but the
+// warp goes on).  Allocation and release are not checked: they sit at fixed,
+// warp-uniform points, and a skipped release would hold the SM's tensor memory
+// and stall the next CTA's allocation.  Release builds compile the check away.
+#ifndef FA_DEBUG
+#define FA_DEBUG 0
+#endif
+__device__ __forceinline__ bool tc_converged(int* err) {
+#if FA_DEBUG
+  if (__activemask() != 0xffffffffu) {
+    if (err) atomicOr(err, kErrDiverged);
+    return false;
+  }
+#else
+  (void)err;
+#endif
+  return true;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -55,7 +81,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Wait until the phase with the given parity of barrier `bar` has completed.
 // Gives up after `limit_ns` of wall time or as soon as *abort is set; on
 // giving up it sets *abort (shared by the CTA) and the device error word and
-// returns false.  No wait in this library can spin forever.
+// returns false.  Every mbarrier wait of the library goes through this bound
+// (or mbar_wait_sleepy's).  It cannot cover the warp-collective tcgen05
+// instructions: those wait inside the hardware for the whole warp, so the
+// kernels keep every branch around them warp-uniform (checked by FA_DEBUG
+// builds, see tc_converged).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           int* err_word, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -120,6 +150,37 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
       : "memory");
+}
+
+// 3-D tiled tensor store shared -> global through a tensor map, tracked by the
+// issuing thread's bulk async-groups.  Elements outside the map's extents are
+// not written.  x must be 16-byte aligned (as for loads); y, z must not be
+// negative.
+__device__ __forceinline__ void tma_store_3d(const void* tmap, uint32_t src, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(tmap)),
+      "r"(src), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+// Contiguous bulk copy shared -> global: both addresses 16-byte aligned, `bytes`
+// a multiple of 16; tracked like tma_store_3d.
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+                   static_cast<uint64_t>(__cvta_generic_to_global(dst))),
+               "r"(src), "r"(bytes)
+               : "memory");
+}
+// Close the thread's current bulk async-group.
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every committed bulk group of this thread has finished reading its
+// shared-memory source (the source may then be overwritten).
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until every committed bulk group of this thread has completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05
@@ -247,7 +308,8 @@ __host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool b_mn_major)
 }
 
 // 32 lanes x 32 bit, 32 consecutive columns per thread (thread i <- lane base+i).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32], int* err) {
+  if (!tc_converged(err)) return;
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -259,7 +321,8 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32], int* err) {
+  if (!tc_converged(err)) return;
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
@@ -271,7 +334,8 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16], int* err) {
+  if (!tc_converged(err)) return;
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
@@ -280,16 +344,19 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[15])
       : "memory");
 }
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8], int* err) {
+  if (!tc_converged(err)) return;
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
       : "memory");
 }
-__device__ __forceinline__ void tmem_wait_ld() {
+__device__ __forceinline__ void tmem_wait_ld(int* err) {
+  if (!tc_converged(err)) return;
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void tmem_wait_st() {
+__device__ __forceinline__ void tmem_wait_st(int* err) {
+  if (!tc_converged(err)) return;
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 

@@ -14,12 +14,14 @@ import re
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libfa_sm100.so")
+# FA_LIBRARY may name another build of the same ABI (e.g. the FA_DEBUG build).
+LIB_PATH = os.environ.get("FA_LIBRARY") or os.path.join(HERE, "libfa_sm100.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "fa.h")
 
 FA_OK = 0
 STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_CUDA",
-          4: "FA_ERR_DEVICE_TIMEOUT", 5: "FA_ERR_DEVICE_INDEX", 6: "FA_ERR_NO_DEVICE"}
+          4: "FA_ERR_DEVICE_TIMEOUT", 5: "FA_ERR_DEVICE_INDEX", 6: "FA_ERR_NO_DEVICE",
+          7: "FA_ERR_DEVICE_DIVERGED"}
 
 _lib = None
 

@@ -49,7 +49,9 @@ enum fa_status {
   FA_ERR_CUDA = 3,           /* a CUDA runtime call or kernel launch failed */
   FA_ERR_DEVICE_TIMEOUT = 4, /* fa_device_status(): a bounded in-kernel wait ran out */
   FA_ERR_DEVICE_INDEX = 5,   /* fa_device_status(): a block-table entry or length was out of range */
-  FA_ERR_NO_DEVICE = 6       /* no sm_100 device is current */
+  FA_ERR_NO_DEVICE = 6,      /* no sm_100 device is current */
+  FA_ERR_DEVICE_DIVERGED = 7 /* fa_device_status(), FA_DEBUG builds only: a tensor-memory
+                                load/store found its warp diverged and was skipped */
 };
 
 /*
@@ -297,13 +299,17 @@ int fa_decode_paged(const void* q, const void* kcache, const void* vcache,
  *
  * Arguments, layouts, supported sizes, outputs and error codes are those of
  * fa_decode_paged.  Differences:
- *   - The partial results need (number of SMs + B) * Hq rows of 516 bytes when
- *     Hkv <= 8 and Hq/Hkv <= 4 (on a 148-SM B200: (148 + B) * Hq <= 32,513), and
- *     B * Hq * chunks
- *     rows otherwise, the chunks being widened until they fit (then the result
- *     agrees with fa_decode_paged within rounding, not bit for bit).  Larger
- *     problems are rejected with FA_ERR_INVALID_ARG before anything touches the
- *     device.
+ *   - The partial results are rows of 516 bytes (128 fp32 values and an LSE).
+ *     With Hkv <= 8 (any supported Hq/Hkv) the persistent schedule needs
+ *     (C + B) * Hq of them plus (B + 2) * 4 bytes of offsets, C being the
+ *     device's SM count: it fits when (C + B) * Hq * 516 + (B + 2) * 4 <=
+ *     16 MiB (C = 148, Hq = 32: B <= 867).
+ *     Problems that it does not fit, and every problem with Hkv > 8, use the
+ *     (chunk, sequence) schedule with B * Hq * chunks rows, the chunks being
+ *     widened until they fit (then the result agrees with fa_decode_paged
+ *     within rounding, not bit for bit).  A problem with B * Hq > 32,513
+ *     (B * Hq * 516 > 16 MiB) fits neither and is rejected with
+ *     FA_ERR_INVALID_ARG before anything touches the device.
  *   - The array is shared by every call and keeps the previous call's contents
  *     (nothing in it needs to start at zero).  Calls whose kernels overlap on
  *     the GPU, e.g. issued on two streams without ordering, race on it.
@@ -311,7 +317,8 @@ int fa_decode_paged(const void* q, const void* kcache, const void* vcache,
  *     loaded, until the process exits.
  *   - The first call on a device looks up the array's device address (once per
  *     device, with that device current); make that first call before any
- *     stream capture.
+ *     stream capture.  After cudaDeviceReset the looked-up address is stale:
+ *     call fa_release() before the next call, which makes it look it up again.
  */
 int fa_decode_paged_noalloc(const void* q, const void* kcache, const void* vcache,
                             const int32_t* block_table, const int32_t* seq_lens, void* o, int B,
@@ -323,12 +330,19 @@ const char* fa_last_error_string(void);
 
 /*
  * Synchronises the current device, then reads and clears its device error
- * word.  Returns FA_OK, FA_ERR_DEVICE_TIMEOUT, FA_ERR_DEVICE_INDEX or
- * FA_ERR_CUDA.
+ * word.  Returns FA_OK, FA_ERR_DEVICE_TIMEOUT, FA_ERR_DEVICE_INDEX,
+ * FA_ERR_DEVICE_DIVERGED (FA_DEBUG builds) or FA_ERR_CUDA; when several bits
+ * are set the first of timeout, divergence, index is reported.
  */
 int fa_device_status(void);
 
-/* Frees the library's cached device resources (decode workspace pools). */
+/*
+ * Frees the library's cached device resources (decode workspace pools, the host
+ * pipeline's streams) and forgets every cached per-device lookup
+ * (device addresses of the library's symbols, kernel attributes), which are
+ * redone on the next call.  Call it after cudaDeviceReset and before using the
+ * library again on that device.  No call of the library may run concurrently.
+ */
 void fa_release(void);
 
 /* Library version: major * 10000 + minor * 100 + patch. */

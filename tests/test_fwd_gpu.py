@@ -72,10 +72,16 @@ def test_small_cases_match_oracle(cuda_device, case):
 
 
 def test_amplified_inputs_within_derived_tolerance(cuda_device):
-    """Values of amplitude 2 and a sharp softmax: exercises the lazy rescale;
-    O is checked against the tolerance derived from the output arithmetic."""
-    check_full(PrefillCase("scale_big", 1, 2, 2, 256, 256, 64, seed=21, scale=0.9, amp=2.0),
-               tol_o=None)
+    """Values of amplitude 2 and a sharp softmax: exercises the lazy rescale.
+    The inputs lie outside the unit-variance workloads the 2e-2 bound is stated
+    for, so O is checked against the bound derived from the output arithmetic
+    (derived_tol_o: 2^-7 max|V|, about 0.07 here); the measured error is printed
+    beside it."""
+    case = PrefillCase("scale_big", 1, 2, 2, 256, 256, 64, seed=21, scale=0.9, amp=2.0)
+    q, k, v, _ = make_prefill(case)
+    dO, dL = check_full(case, tol_o=None)
+    print(f"scale_big: max|dO| = {dO:.3e} against the derived bound {derived_tol_o(v):.3e}; "
+          f"max|dLSE| = {dL:.3e}")
 
 
 def test_tiny_workload(cuda_device):
@@ -103,8 +109,11 @@ def check_sampled(case, per_head):
     assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
 
 
-def test_llama3_8b_gqa_causal_workload_sampled(cuda_device):
-    check_sampled(PREFILL_CASES["gqa_b1_hq32_hkv8_n8192_d128_causal"], 16)
+def test_llama3_8b_gqa_causal_workload_full_compare(cuda_device):
+    """Every one of the 262,144 output rows (32 heads x 8192 queries) against the
+    oracle's materialised-score attention, element by element."""
+    dO, dL = check_full(PREFILL_CASES["gqa_b1_hq32_hkv8_n8192_d128_causal"])
+    print(f"gqa_b1_hq32_hkv8_n8192_d128_causal: max|dO| = {dO:.3e}, max|dLSE| = {dL:.3e}")
 
 
 def test_long_context_131072_workload_sampled(cuda_device):
