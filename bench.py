@@ -15,6 +15,12 @@ and divided by the slowest rank's prefill time; the decode KV GB/s is reported
 beside it.  Multi-GPU runs are weak-scaled replicas (each rank runs the same
 per-rank workload on its own inputs; the path has no exchange step).
 
+Rows beyond the headline (``"widened"``, rank 0 at N=1, timed outside the
+headline's region, each with its roofline fraction): ragged and paged prefill,
+the (2, 8, 4096, 64) fp16 workload with and without the causal mask, the
+131072-token causal GQA workload, the FP8 forward and its quantiser, and the
+backward.  ``--headline-only`` skips them.
+
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
 workloads (rank 0 only).
 """
@@ -308,10 +314,9 @@ def widened_rows(fa, dev, stream, flush, warmup, steps, peaks, peak_src):
     return out
 
 
-def pending_rows(fa, dev, stream, flush, warmup, steps, peaks, peak_src):
-    """Kernels built but not yet verified on a B200 (FP8 forward and its
-    quantiser, backward): timed on the headline prefill workload only when
-    --pending is given, never in a default run."""
+def fp8_and_backward_rows(fa, dev, stream, flush, warmup, steps, peaks, peak_src):
+    """The FP8 forward and its quantiser, and the backward, on the headline
+    prefill workload (B1 Hq32 Hkv8 N8192 D128 causal), each with its roofline."""
     from exact_tiled_attention_40_b200.inputs import FP8_CASES, hadamard_signs, make_dout
     out = {}
     sp = stream.cuda_stream
@@ -384,6 +389,92 @@ def pending_rows(fa, dev, stream, flush, warmup, steps, peaks, peak_src):
     return out
 
 
+def oracle_heads_sample(case, heads: int = 1):
+    """fp64 oracle on the first `heads` query heads of batch entry 0 of a dense
+    prefill workload (full rows).  Returns (TFLOP/s, seconds, sample text)."""
+    import oracle
+    q, k, v, _ = make_prefill(case)
+    g = case.Hq // case.Hkv
+    hk = max(1, -(-heads // g))
+    qs = q[:1, :heads].float().double().numpy()
+    ks = k[:1, :hk].float().double().numpy()
+    vs = v[:1, :hk].float().double().numpy()
+    t0 = time.perf_counter()
+    oracle.attention(qs, ks, vs, case.softmax_scale, case.causal)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * heads * case.Nq * case.Nk * case.D / (2 if case.causal else 1)
+    return flops / dt / 1e12, dt, f"{heads} of {case.B * case.Hq} (sequence, head) pairs of {case.name}, fp64"
+
+
+def oracle_rows_sample(case, rows: int = 8):
+    """fp64 oracle on `rows` query rows of head 0 (the last rows, full causal
+    prefixes) of a long workload.  Returns (TFLOP/s, seconds, sample text)."""
+    import oracle
+    q, k, v, _ = make_prefill(case)
+    sel = [(0, 0, case.Nq - 1 - r) for r in range(rows)]
+    kd = k[:, :1].float().double().numpy()
+    vd = v[:, :1].float().double().numpy()
+    qd = q[:, :1].float().double().numpy()
+    t0 = time.perf_counter()
+    oracle.attention_rows(qd, kd, vd, case.softmax_scale, case.causal, sel)
+    dt = time.perf_counter() - t0
+    flops = sum(4.0 * (i + 1) * case.D for _, _, i in sel)
+    return flops / dt / 1e12, dt, f"{rows} query rows (full causal prefixes) of {case.name}, fp64"
+
+
+def dense_prefill_rows(fa, dev, stream, flush, warmup, steps, peaks, peak_src):
+    """The pages' other dense prefill workloads: (2, 8, 4096, 64) fp16 with and
+    without the causal mask, and the 131072-token causal GQA case."""
+    out = {}
+    sp = stream.cuda_stream
+    specs = [("mha_fp16", "mha_b2_h8_n4096_d64_fp16", oracle_heads_sample),
+             ("mha_fp16_causal", "mha_b2_h8_n4096_d64_fp16_causal", oracle_heads_sample),
+             ("long_context", "gqa_b1_hq32_hkv8_n131072_d128_causal", oracle_rows_sample)]
+    for key, name, sample_fn in specs:
+        c = PREFILL_CASES[name]
+        try:
+            q_h, k_h, v_h, _ = make_prefill(c)
+            q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+            del q_h, k_h, v_h
+            o = torch.empty_like(q)
+            lse = torch.empty((c.B, c.Hq, c.Nq), dtype=torch.float32, device=dev)
+            long_case = c.Nq > 16384
+            n_warm, n_steps = (3, 5) if long_case else (warmup, steps)
+            ts = []
+            for i in range(n_warm + n_steps):
+                flush.fill_(i & 0xff)
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fa.fa_fwd(q, k, v, o, lse, c.B, c.Hq, c.Hkv, c.Nq, c.Nk, c.D, c.softmax_scale,
+                          c.causal, stream=sp)
+                b.record(stream)
+                b.synchronize()
+                if i >= n_warm:
+                    ts.append(a.elapsed_time(b))
+            if fa.device_status() != 0:
+                raise RuntimeError(fa.last_error())
+            ms = statistics.median(ts)
+            tf = c.flops / (ms * 1e-3) / 1e12
+            otf, odt, sample = sample_fn(c)
+            out[key] = {"workload": c.name, "dtype": c.dtype, "value": tf, "unit": "TFLOP/s",
+                        "ms_per_launch": ms, "launches_timed": n_steps,
+                        "roofline": {"bound": "tensor", "achieved": tf,
+                                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                     "frac": tf / peaks["bf16_tflops"],
+                                     "peak_source": f"{peak_src} burst bf16 (fp16 dense "
+                                                    "tensor peak is the same)",
+                                     "frac_of_nominal_2250": tf / 2250.0},
+                        "cpu_baseline": {"value": otf, "unit": "TFLOP/s",
+                                         "cores": cpu_threads(), "kind": "oracle",
+                                         "sample": sample, "seconds": odt}}
+            del q, k, v, o, lse
+            torch.cuda.empty_cache()
+        except Exception as e:  # reported, never fatal for the headline line
+            out[key] = {"workload": c.name, "error": f"{type(e).__name__}: {e}"[:300]}
+    return out
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return 0
@@ -420,8 +511,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pending", action="store_true",
-                    help="also time the kernels that await their first B200 verification")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the rows beyond the headline prefill and decode")
     args = ap.parse_args()
     world, rank, local = dist_env()
     if args.impl == "reference":
@@ -605,12 +696,16 @@ def main():
         tf, dt, sample = oracle_prefill_sample(heads=8)
         line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cpu_threads(),
                                 "kind": "oracle", "sample": sample, "seconds": dt}
+    if rank == 0 and world == 1 and not args.headline_only:
         # rows beyond the headline path, measured outside its timed region
-        line["widened"] = widened_rows(fa, dev, stream, flush, args.warmup, min(args.steps, 10),
-                                       peaks, peak_src)
-    if rank == 0 and world == 1 and args.pending:
-        line["pending"] = pending_rows(fa, dev, stream, flush, args.warmup, min(args.steps, 10),
-                                       peaks, peak_src)
+        del q, k, v, o, lse, dq, kc, vc, table, lens, do, dlse
+        torch.cuda.empty_cache()
+        n = min(args.steps, 10)
+        line["widened"] = widened_rows(fa, dev, stream, flush, args.warmup, n, peaks, peak_src)
+        line["widened"].update(dense_prefill_rows(fa, dev, stream, flush, args.warmup, n, peaks,
+                                                  peak_src))
+        line["widened"].update(fp8_and_backward_rows(fa, dev, stream, flush, args.warmup, n,
+                                                     peaks, peak_src))
     if rank == 0:
         print(json.dumps(line), flush=True)
     if pg is not None:

@@ -64,22 +64,29 @@ static_assert(kRegsControl * 128 + kRegsSoftmax * 256 <= 384 * 168, "register sp
 
 constexpr int kSchedMax = 2048;   // entries of the work-sorted list of ragged batches
 
-// SCHED: the ragged and paged kernels also keep their work-sorted (pair,
-// sequence) list in shared memory, and give up one K/V slot at D = 128 for it.
+// SCHED: the ragged and paged kernels keep their work-sorted (pair, sequence)
+// list in shared memory.  The dense kernel instead stages its epilogue there:
+// per softmax warp a 32-row x 64-column bf16/fp16 box of O (4 KB, laid out as
+// the 128-byte swizzle of the O tensor map) and the warp's 32 LSE values, which
+// the TMA engine writes to global memory.
 template <int D, bool SCHED = false>
 struct FwdLayout {
   static constexpr int kChunks = D / 64;              // 128-byte swizzle atoms along D
   static constexpr int kChunkBytes = kBM * 128;       // one atom column of a 128-row tile
   static constexpr int kTileBytes = kBM * D * 2;      // a 128-row tile of Q, K or V
-  static constexpr int kSlots = D == 128 ? (SCHED ? 4 : 5) : 8;   // K/V ring slots
+  static constexpr int kSlots = D == 128 ? 4 : 8;     // K/V ring slots
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
   static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 4 + 2 + 1 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;   // tmem address, abort, list size, ok
   static constexpr int kSchedOff = kMiscOff + 16;
+  static constexpr int kStageOBytes = 32 * 128;              // one warp's O box
+  static constexpr int kStageOff = (kSchedOff + 1023) & ~1023;   // swizzle atoms: 1024-aligned
+  static constexpr int kStageLseOff = kStageOff + 8 * kStageOBytes;
   static constexpr int kSmemBytes =
-      kSchedOff + (SCHED ? kSchedMax * 4 : 0) + 1024;     // + slack for 1024-byte alignment
+      (SCHED ? kSchedOff + kSchedMax * 4 : kStageLseOff + 8 * 32 * 4) +
+      1024;                                                  // + slack for 1024-byte alignment
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -102,6 +109,7 @@ struct FwdParams {
   int num_mpairs;
   int num_items;      // num_mpairs * B * Hq work items, heaviest first
   int causal;
+  int lse_bulk;       // dense: LSE rows leave by bulk copies (Nq % 4 == 0, lse 16-byte aligned)
   float scale_log2;   // scale * log2(e)
   int* err;
   uint64_t timeout_ns;
@@ -276,7 +284,8 @@ struct ItemWalker {
 template <int D, bool BF16, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                  const FwdParams p) {
   constexpr bool RAGGED = MODE != kDense;
   using L = FwdLayout<D, RAGGED>;
   extern __shared__ uint8_t smem_raw[];
@@ -762,29 +771,87 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         tc_fence_after();
         const float inv_l = l > 0.f ? 1.f / l : 0.f;
+        const float lse_v =
+            l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+        if constexpr (MODE == kDense) {
+          // TMA epilogue.  Per 64-column half, the warp's 32 rows go to its
+          // staging box (128-byte swizzle: 16-byte chunk k of row r at k ^ (r & 7),
+          // conflict-free), then one lane stores the box through the O tensor map,
+          // which clips rows past Nq; the LSE values leave by one bulk copy.
+          const uint32_t stage = sbase + L::kStageOff + warp * L::kStageOBytes;
+          const int row0 = tile_first + (warp & 3) * 32;   // the warp's first row
+          const bool slab_live = row0 < it.nq;              // warp-uniform
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t ov[32];
-          tmem_ld32(tO + 32 * c, ov, p.err);
-          tmem_wait_ld(p.err);
-          uint32_t pk[16];
+          for (int hh = 0; hh < D / 64; ++hh) {
+            if (lane == 0) bulk_wait_read_all();   // earlier boxes have left the stage
+            __syncwarp();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float a = __uint_as_float(ov[2 * e]) * inv_l;
-            const float bb = __uint_as_float(ov[2 * e + 1]) * inv_l;
-            pk[e] = BF16 ? pack_bf16x2(a, bb) : pack_f16x2(a, bb);
-          }
-          if (row < it.nq) {
-            uint4* dst = reinterpret_cast<uint4*>(o_row + 32 * c);
+            for (int cc = 0; cc < 2; ++cc) {
+              uint32_t ov[32];
+              tmem_ld32(tO + 64 * hh + 32 * cc, ov, p.err);
+              tmem_wait_ld(p.err);
+              uint32_t pk[16];
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+              for (int e = 0; e < 16; ++e) {
+                const float a = __uint_as_float(ov[2 * e]) * inv_l;
+                const float bb = __uint_as_float(ov[2 * e + 1]) * inv_l;
+                pk[e] = BF16 ? pack_bf16x2(a, bb) : pack_f16x2(a, bb);
+              }
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                st_shared_v4(stage + lane * 128 + (((cc * 4 + v) ^ (lane & 7)) << 4), pk[4 * v],
+                             pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && slab_live) {
+              tma_store_3d(&tmO, stage, 64 * hh, row0, it.bh);
+              bulk_commit();
+            }
           }
+          if (p.lse) {
+            if (p.lse_bulk) {
+              const uint32_t lst = sbase + L::kStageLseOff + warp * 128;
+              st_shared_f32(lst + lane * 4, lse_v);
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0 && slab_live) {
+                const int nrows = min(32, it.nq - row0);   // a multiple of 4 (Nq % 4 == 0)
+                bulk_store(p.lse + static_cast<size_t>(it.bh) * p.Nq + row0, lst, nrows * 4);
+                bulk_commit();
+              }
+            } else if (row < it.nq) {
+              p.lse[row_index] = lse_v;
+            }
+          }
+        } else {
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(tO + 32 * c, ov, p.err);
+            tmem_wait_ld(p.err);
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float a = __uint_as_float(ov[2 * e]) * inv_l;
+              const float bb = __uint_as_float(ov[2 * e + 1]) * inv_l;
+              pk[e] = BF16 ? pack_bf16x2(a, bb) : pack_f16x2(a, bb);
+            }
+            if (row < it.nq) {
+              uint4* dst = reinterpret_cast<uint4*>(o_row + 32 * c);
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            }
+          }
+          if (p.lse && row < it.nq) p.lse[row_index] = lse_v;
         }
-        if (p.lse && row < it.nq)
-          p.lse[row_index] = l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
       }
     }
+    }
+    // the stores of the last epilogue complete before the CTA's shared memory goes
+    if constexpr (MODE == kDense) {
+      if (lane == 0) bulk_wait_all();
     }
   }
 
@@ -806,6 +873,16 @@ int encode_3d(CUtensorMap* m, const void* base, bool bf16, int D, int N, int Z) 
   const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2,
                                static_cast<uint64_t>(N) * static_cast<uint64_t>(D) * 2};
   const uint32_t box[3] = {64, 128, 1};
+  return encode_tensor_map_16bit(m, base, bf16, 3, dims, strides, box);
+}
+// Store map of the dense output O [Z, N, D]: a 64 x 32 x 1 box (one softmax
+// warp's rows, one swizzle atom column) with 128-byte swizzle.
+int encode_o_store(CUtensorMap* m, void* base, bool bf16, int D, int N, int Z) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(N),
+                            static_cast<uint64_t>(Z)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2,
+                               static_cast<uint64_t>(N) * static_cast<uint64_t>(D) * 2};
+  const uint32_t box[3] = {64, 32, 1};
   return encode_tensor_map_16bit(m, base, bf16, 3, dims, strides, box);
 }
 // 3-D map over a packed [T, H, D] tensor (token-major) with a 64 x 1 x rows box:
@@ -884,9 +961,12 @@ int launch_typed(const void* q, const void* k, const void* v, void* o, float* ls
     tk = tq;   // no key tile exists, so these maps are never read
     tv = tq;
   }
+  CUtensorMap to = tq;   // ragged and paged batches store O with plain stores
+  if (!cu_q && (rc = encode_o_store(&to, o, BF16, D, Nq, B * Hq)) != FA_OK) return rc;
   FwdParams prm;
   prm.o = o;
   prm.lse = lse;
+  prm.lse_bulk = lse != nullptr && (Nq % 4) == 0 && (reinterpret_cast<uintptr_t>(lse) & 15u) == 0;
   prm.cu_q = cu_q;
   prm.cu_k = la.cu_k;
   prm.total_q = total_q;
@@ -916,11 +996,11 @@ int launch_typed(const void* q, const void* k, const void* v, void* o, float* ls
   if (grid == 0) return FA_OK;
   const unsigned g = static_cast<unsigned>(grid);
   if (paged)
-    fa_fwd_kernel<D, BF16, kPaged><<<g, kThreads, LR::kSmemBytes, stream>>>(tq, tk, tv, prm);
+    fa_fwd_kernel<D, BF16, kPaged><<<g, kThreads, LR::kSmemBytes, stream>>>(tq, tk, tv, to, prm);
   else if (cu_q)
-    fa_fwd_kernel<D, BF16, kRagged><<<g, kThreads, LR::kSmemBytes, stream>>>(tq, tk, tv, prm);
+    fa_fwd_kernel<D, BF16, kRagged><<<g, kThreads, LR::kSmemBytes, stream>>>(tq, tk, tv, to, prm);
   else
-    fa_fwd_kernel<D, BF16, kDense><<<g, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, prm);
+    fa_fwd_kernel<D, BF16, kDense><<<g, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, to, prm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(FA_ERR_CUDA, "fa_fwd launch: %s", cudaGetErrorString(e));
   return FA_OK;

@@ -52,21 +52,31 @@ def f64(t):
     return t.float().double().cpu().numpy()
 
 
-def test_forward_touches_nothing_outside_its_tensors(cuda_device):
-    case = PrefillCase("canary_fwd", 2, 4, 2, 300, 300, 128, seed=120, causal=True)
+FP16_NAN = 0x7E01                # an fp16 NaN, as int16 bits
+
+
+@pytest.mark.parametrize("case", [
+    # rows past Nq = 300 in the last query tile: the O tensor map clips them; LSE rows
+    # leave by bulk copies (Nq % 4 == 0)
+    PrefillCase("canary_fwd", 2, 4, 2, 300, 300, 128, seed=120, causal=True),
+    # fp16, D = 64, Nq = 77 (not a multiple of 4: LSE by plain stores), more keys than queries
+    PrefillCase("canary_fwd_fp16", 2, 2, 1, 77, 390, 64, "fp16", seed=122),
+], ids=lambda c: c.name)
+def test_forward_touches_nothing_outside_its_tensors(cuda_device, case):
     q, k, v, _ = make_prefill(case)
     dev = cuda_device
-    gq = Guarded(q.shape, torch.bfloat16, dev, BF16_NAN, q)
-    gk = Guarded(k.shape, torch.bfloat16, dev, BF16_NAN, k)
-    gv = Guarded(v.shape, torch.bfloat16, dev, BF16_NAN, v)
-    go = Guarded(q.shape, torch.bfloat16, dev, OUT_BITS16)
+    dt, nan = (torch.bfloat16, BF16_NAN) if case.dtype == "bf16" else (torch.float16, FP16_NAN)
+    gq = Guarded(q.shape, dt, dev, nan, q)
+    gk = Guarded(k.shape, dt, dev, nan, k)
+    gv = Guarded(v.shape, dt, dev, nan, v)
+    go = Guarded(q.shape, dt, dev, OUT_BITS16)
     gl = Guarded((case.B, case.Hq, case.Nq), torch.float32, dev, OUT_BITS32)
     fa.fa_fwd(gq.t, gk.t, gv.t, go.t, gl.t, case.B, case.Hq, case.Hkv, case.Nq, case.Nk, case.D,
-              case.softmax_scale, True)
+              case.softmax_scale, case.causal)
     torch.cuda.synchronize()
     assert fa.device_status() == 0, fa.last_error()
     assert go.margins_intact() and gl.margins_intact()
-    O, L = oracle.attention(f64(q), f64(k), f64(v), case.softmax_scale, True)
+    O, L = oracle.attention(f64(q), f64(k), f64(v), case.softmax_scale, case.causal)
     assert np.abs(f64(go.t) - O).max() <= 2e-2
     assert np.abs(f64(gl.t) - L).max() <= 1e-3
 
