@@ -42,7 +42,10 @@ namespace fa {
 namespace {
 
 constexpr int kBM = 128;                  // rows of every tile (TMEM lanes)
-constexpr int kThreads = 192;             // 4 softmax warps, producer, MMA
+constexpr int kHalfN = 64;                // columns of a softmax warpgroup's half tile
+constexpr int kThreads = 320;             // 2 x 4 softmax warps, producer, MMA
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
@@ -54,12 +57,17 @@ struct BwdLayout {
   static constexpr int kFixOff = 0;
   static constexpr int kRingOff = 2 * kTileBytes;
   static constexpr int kBarOff = kRingOff + 4 * kTileBytes;
-  static constexpr int kNumBars = 1 + 2 + 2 + 1 + 1 + 1;
+  static constexpr int kNumBars = 1 + 2 + 2 + 2 + 2 + 1 + 4;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  // dK/dV kernel: per warpgroup and item parity, the 64 queries' LSE (log2
+  // units) and delta
+  static constexpr int kStatOff = kMiscOff + 16;
+  static constexpr int kStatBytes = 2 * 2 * 2 * kHalfN * 4;
   // at least 118 KB so that two CTAs never share an SM: each allocates all 512
   // TMEM columns (the next power of two above its 384 or 320 at D = 64)
-  static constexpr int kSmemBytes =
-      (kMiscOff + 16 + 1024) > 118 * 1024 ? (kMiscOff + 16 + 1024) : 118 * 1024;
+  static constexpr int kSmemBytes = (kStatOff + kStatBytes + 1024) > 118 * 1024
+                                        ? (kStatOff + kStatBytes + 1024)
+                                        : 118 * 1024;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -117,43 +125,46 @@ __device__ __forceinline__ uint64_t kmajor_step(int kk) {
   return static_cast<uint64_t>(((kk >> 2) * BwdLayout<D>::kChunkBytes + (kk & 3) * 32) >> 4);
 }
 
-// 128 x 128 product of two K-major [128, D] tiles (rows of A against rows of B)
-// into TMEM columns d .. d + 127.
+// 128 x 64 product of two K-major [128, D] tiles: rows of A against rows
+// row0 .. row0 + 63 of B (row0 a multiple of 64: a whole number of 8-row
+// swizzle atoms), into TMEM columns d .. d + 63.
 template <int D>
-__device__ __forceinline__ void mma_rows_x_rows(uint32_t d, uint64_t a, uint64_t b) {
-  constexpr uint32_t idesc = idesc_f16(kBM, kBM, true, false);
+__device__ __forceinline__ void mma_rows_x_half(uint32_t d, uint64_t a, uint64_t b, int row0) {
+  constexpr uint32_t idesc = idesc_f16(kBM, kHalfN, true, false);
+  const uint64_t boff = static_cast<uint64_t>((row0 * 128) >> 4);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk)
-    mma_ss(d, a + kmajor_step<D>(kk), b + kmajor_step<D>(kk), idesc, kk > 0 ? 1u : 0u);
+    mma_ss(d, a + kmajor_step<D>(kk), b + boff + kmajor_step<D>(kk), idesc, kk > 0 ? 1u : 0u);
 }
 
-// D-column accumulation: TMEM[d .. d + D) (+)= A (bf16 pairs in TMEM columns
-// a .. a + 63, 128 K values) x B ([128, D] tile read MN-major).
+// D-column accumulation over 64 K values k0 .. k0 + 63: TMEM[d .. d + D) (+)=
+// A (bf16 pairs in TMEM columns a .. a + 31) x B (rows k0 .. of a [128, D]
+// tile, read MN-major).
 template <int D>
-__device__ __forceinline__ void mma_tmem_x_tile(uint32_t d, uint32_t a, uint64_t b_mn,
+__device__ __forceinline__ void mma_half_x_tile(uint32_t d, uint32_t a, uint64_t b_mn, int k0,
                                                 bool accumulate) {
   constexpr uint32_t idesc = idesc_f16(kBM, D, true, true);
 #pragma unroll
-  for (int kk = 0; kk < kBM / 16; ++kk)
-    mma_ts(d, a + kk * 8, b_mn + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc,
-           (accumulate || kk > 0) ? 1u : 0u);
+  for (int k = 0; k < kHalfN / 16; ++k)
+    mma_ts(d, a + k * 8, b_mn + static_cast<uint64_t>(((k0 + k * 16) * 128) >> 4), idesc,
+           (accumulate || k > 0) ? 1u : 0u);
 }
 
-// Store a row of D fp32 TMEM values (columns t0 ..), times `mul`, as bf16.
-template <int D>
-__device__ __forceinline__ void store_row_bf16(uint32_t t0, float mul, uint16_t* dst, bool valid,
-                                               int* err) {
+// Store columns c0 .. c0 + ncols of a row of fp32 TMEM values (columns t0 ..),
+// times `mul`, as bf16 (32 columns per step).
+__device__ __forceinline__ void store_cols_bf16(uint32_t t0, int c0, int ncols, float mul,
+                                                uint16_t* dst, bool valid, int* err) {
 #pragma unroll 1
-  for (int c = 0; c < D / 32; ++c) {
+  for (int c = c0; c < c0 + ncols; c += 32) {
     uint32_t v[32];
-    tmem_ld32(t0 + 32 * c, v, err);
+    tmem_ld32(t0 + c, v, err);
     tmem_wait_ld(err);
     uint32_t pk[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e)
       pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
     if (valid) {
-      uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+      uint4* d4 = reinterpret_cast<uint4*>(dst + c);
 #pragma unroll
       for (int q = 0; q < 4; ++q)
         d4[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
@@ -161,11 +172,9 @@ __device__ __forceinline__ void store_row_bf16(uint32_t t0, float mul, uint16_t*
   }
 }
 
-template <int D>
-__device__ __forceinline__ void store_zero_row(uint16_t* dst) {
+__device__ __forceinline__ void store_zero_cols(uint16_t* dst, int c0, int ncols) {
   const uint4 z = make_uint4(0, 0, 0, 0);
-#pragma unroll
-  for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(dst)[c] = z;
+  for (int c = c0; c < c0 + ncols; c += 8) *reinterpret_cast<uint4*>(dst + c) = z;
 }
 
 // First query tile that sees key tile j (causal, bottom-right aligned).
@@ -176,6 +185,13 @@ __device__ __forceinline__ int first_q_tile(int j, int Nq, int Nk, int causal) {
 }
 
 // ---------------------------------------------------------------- dK, dV
+// Warps 0-3 and 4-7 are two softmax warpgroups over the same 128 TMEM lanes
+// (key rows): warpgroup w takes the queries 64 w .. 64 w + 63 of each tile
+// pair, i.e. columns 64 w .. of S^T and 128 + 64 w .. of dP^T, and writes its
+// P^T and dS^T there as 32 columns of bf16 pairs.  The MMA warp computes each
+// half of S^T and dP^T with N = 64 MMAs and commits the halves separately, so
+// warpgroup 0 starts while the second half is computed; dV and dK take each
+// half's 64 queries as soon as its warpgroup has released it.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -209,11 +225,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t kv_full = bar(0);
   auto q_full = [&](int s) { return bar(1 + s); };
   auto q_empty = [&](int s) { return bar(3 + s); };
-  const uint32_t s_full = bar(5);
-  const uint32_t p_full = bar(6);
-  const uint32_t acc_done = bar(7);
+  auto s_full = [&](int h) { return bar(5 + h); };
+  auto p_full = [&](int h) { return bar(7 + h); };
+  const uint32_t acc_done = bar(9);
+  // a warpgroup's staged LSE and delta of one item parity are complete
+  auto stat_full = [&](int w, int par) { return bar(10 + 2 * w + par); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  float* stat = reinterpret_cast<float*>(smem + L::kStatOff);
   const uint32_t k_smem = sbase + L::kFixOff;
   const uint32_t v_smem = sbase + L::kFixOff + L::kTileBytes;
   auto q_smem = [&](int s) { return sbase + L::kRingOff + (2 * s) * L::kTileBytes; };
@@ -224,14 +243,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(q_full(s), 1);
       mbar_init(q_empty(s), 1);
+      mbar_init(s_full(s), 1);
+      mbar_init(p_full(s), kBM);
+      mbar_init(stat_full(s, 0), kBM);
+      mbar_init(stat_full(s, 1), kBM);
     }
-    mbar_init(s_full, 1);
-    mbar_init(p_full, kBM);
     mbar_init(acc_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -239,10 +260,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // TMEM: [0,128) S^T then P^T (bf16 pairs in [0,64)); [128,256) dP^T then dS^T;
-  // [256,256+D) dV; [256+D,256+2D) dK
+  // TMEM: [0,128) S^T then P^T (warpgroup w's bf16 pairs in [64w, 64w+32));
+  // [128,256) dP^T then dS^T likewise; [256,256+D) dV; [256+D,256+2D) dK
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && n_items > 0) {
       tma_prefetch_desc(&tmQ);
@@ -276,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(q_full(s), (last >> 1) & 1, &no_abort, p.err, p.timeout_ns);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     const bool leader = elect_one();
     auto wait = [&](uint32_t br, uint32_t parity) {
@@ -293,70 +314,96 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t q_kdesc = smem_desc_sw128(q_smem(s), 16, 1024);
       const uint64_t do_kdesc = smem_desc_sw128(do_smem(s), 16, 1024);
       if (leader) {
-        mma_rows_x_rows<D>(tmem + 0, k_desc, q_kdesc);       // S^T = K_j Q_i^T
-        mma_rows_x_rows<D>(tmem + 128, v_desc, do_kdesc);    // dP^T = V_j dO_i^T
-        tc_commit(s_full);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          mma_rows_x_half<D>(tmem + kHalfN * h, k_desc, q_kdesc, kHalfN * h);          // S^T
+          mma_rows_x_half<D>(tmem + 128 + kHalfN * h, v_desc, do_kdesc, kHalfN * h);   // dP^T
+          tc_commit(s_full(h));
+        }
       }
-      ok = wait(p_full, it & 1);
-      if (!ok) break;
-      tc_fence_after();
       const uint64_t q_mn = smem_desc_sw128(q_smem(s), L::kChunkBytes, 1024);
       const uint64_t do_mn = smem_desc_sw128(do_smem(s), L::kChunkBytes, 1024);
-      if (leader) {
-        mma_tmem_x_tile<D>(tmem + 256, tmem + 0, do_mn, it > 0);        // dV += P^T dO_i
-        mma_tmem_x_tile<D>(tmem + 256 + D, tmem + 128, q_mn, it > 0);   // dK += dS^T Q_i
-        tc_commit(q_empty(s));
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        ok = wait(p_full(h), it & 1);
+        if (!ok) break;
+        tc_fence_after();
+        if (leader) {
+          const bool acc = it > 0 || h > 0;
+          mma_half_x_tile<D>(tmem + 256, tmem + kHalfN * h, do_mn, kHalfN * h, acc);        // dV
+          mma_half_x_tile<D>(tmem + 256 + D, tmem + 128 + kHalfN * h, q_mn, kHalfN * h, acc);  // dK
+        }
       }
+      if (!ok) break;
+      if (leader) tc_commit(q_empty(s));
     }
     if (leader) tc_commit(acc_done);
     volatile int no_abort = 0;
     mbar_wait(acc_done, 0, &no_abort, p.err, p.timeout_ns);
   } else {
-    // ------------------------------------------------------------ softmax warpgroup
-    const int r = tid;                                  // key row within the tile
+    // ------------------------------------------------------------ softmax warpgroups
+    const int wg = warp >> 2;                           // queries 64 wg .. 64 wg + 63
+    const int t = tid & 127;
+    const int r = (warp & 3) * 32 + lane;               // key row within the tile
     const int kr = j * kBM + r;                         // key index
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_base;
-    const uint32_t tP = tmem + lane_base + 128;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + kHalfN * wg;
+    const uint32_t tP = tmem + lane_base + 128 + kHalfN * wg;
     bool ok = true;
     for (int it = 0; ok && it < n_items; ++it) {
       const int g = it / per_head;
       const int i = i0 + (it - g * per_head);
       const size_t qrow0 = static_cast<size_t>(b * p.Hq + hkv * G + g) * p.Nq;
-      const bool got = mbar_wait(s_full, it & 1, abort_flag, p.err, p.timeout_ns);
+      const int q0 = i * kBM + kHalfN * wg;            // first query of this half
+      // the half's 64 LSE (log2 units) and delta values, staged once per item in
+      // a buffer of this item's parity (the buffer of item it - 2 is free: every
+      // thread of the warpgroup has passed item it - 1's stat barrier)
+      float* lse2_s = stat + ((wg * 2 + (it & 1)) * 2) * kHalfN;
+      float* dl_s = lse2_s + kHalfN;
+      {
+        const int q = q0 + (t & 63);
+        if (t < 64)
+          lse2_s[t] = q < p.Nq ? __ldg(p.lse + qrow0 + q) * kLog2e : INFINITY;
+        else
+          dl_s[t - 64] = q < p.Nq ? __ldg(p.delta + qrow0 + q) : 0.f;
+      }
+      mbar_arrive(stat_full(wg, it & 1));
+      bool got = mbar_wait(stat_full(wg, it & 1), (it >> 1) & 1, abort_flag, p.err, p.timeout_ns);
+      if (got) got = mbar_wait(s_full(wg), it & 1, abort_flag, p.err, p.timeout_ns);
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      // queries q0 + e of this chunk are visible to key kr when kr <= q + off
-      const bool band = p.causal && (j * kBM + kBM - 1 > i * kBM + off);
+      // queries q0 + e are visible to key kr when kr <= q + off
+      const bool band = p.causal && (j * kBM + kBM - 1 > q0 + off);
+      const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t sv[32], dv[32];
         tmem_ld32(tS + 32 * c, sv, p.err);
         tmem_ld32(tP + 32 * c, dv, p.err);
         tmem_wait_ld(p.err);
-        const int q0 = i * kBM + 32 * c;
         uint32_t pk[16], dk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          float pe[2], de[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int q = q0 + e + u;
-            float lse = INFINITY, dl = 0.f;
-            if (q < p.Nq) {
-              lse = __ldg(p.lse + qrow0 + q);
-              dl = __ldg(p.delta + qrow0 + q);
-            }
-            float pv = ex2(fmaf(__uint_as_float(sv[e + u]), p.scale_log2, -lse * kLog2e));
-            if (band && kr > q + off) pv = 0.f;
-            pe[u] = pv;
-            de[u] = pv * (__uint_as_float(dv[e + u]) - dl);
+          const int ee = 32 * c + e;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), c2,
+                           f2_pack(-lse2_s[ee], -lse2_s[ee + 1])),
+                    x0, x1);
+          float p0 = ex2(x0), p1 = ex2(x1);
+          if (band) {
+            if (kr > q0 + ee + off) p0 = 0.f;
+            if (kr > q0 + ee + 1 + off) p1 = 0.f;
           }
-          pk[e >> 1] = pack_bf16x2(pe[0], pe[1]);
-          dk[e >> 1] = pack_bf16x2(de[0], de[1]);
+          float d0, d1;
+          f2_unpack(f2_mul(f2_pack(p0, p1),
+                           f2_sub(f2_pack(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])),
+                                  f2_pack(dl_s[ee], dl_s[ee + 1]))),
+                    d0, d1);
+          pk[e >> 1] = pack_bf16x2(p0, p1);
+          dk[e >> 1] = pack_bf16x2(d0, d1);
         }
         // the packed pairs go over columns already read (16 c .. 16 c + 15)
         tmem_st16(tS + 16 * c, pk, p.err);
@@ -364,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tmem_wait_st(p.err);
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(p_full(wg));
     }
     const bool fin = ok && (n_items == 0 ||
                             mbar_wait(acc_done, 0, abort_flag, p.err, p.timeout_ns));
@@ -372,21 +419,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const size_t orow = (static_cast<size_t>(b * p.Hkv + hkv) * p.Nk + kr) * D;
       const bool valid = kr < p.Nk;
+      const int c0 = wg * (D / 2);                     // this warpgroup's half of the columns
       if (n_items == 0) {
         if (valid) {
-          store_zero_row<D>(p.dv + orow);
-          store_zero_row<D>(p.dk + orow);
+          store_zero_cols(p.dv + orow, c0, D / 2);
+          store_zero_cols(p.dk + orow, c0, D / 2);
         }
       } else {
-        store_row_bf16<D>(tmem + lane_base + 256, 1.f, p.dv + orow, valid, p.err);
-        store_row_bf16<D>(tmem + lane_base + 256 + D, p.scale, p.dk + orow, valid, p.err);
+        store_cols_bf16(tmem + lane_base + 256, c0, D / 2, 1.f, p.dv + orow, valid, p.err);
+        store_cols_bf16(tmem + lane_base + 256 + D, c0, D / 2, p.scale, p.dk + orow, valid,
+                        p.err);
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -394,6 +443,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- dQ
+// Two softmax warpgroups over the same 128 query rows: warpgroup w takes keys
+// 64 w .. 64 w + 63 of each key tile (columns 64 w .. of S and 128 + 64 w .. of
+// dP) and writes its dS there as 32 columns of bf16 pairs; dQ takes each
+// half's keys as soon as its warpgroup has released it.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -429,9 +482,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t q_full = bar(0);
   auto kv_full = [&](int s) { return bar(1 + s); };
   auto kv_empty = [&](int s) { return bar(3 + s); };
-  const uint32_t s_full = bar(5);
-  const uint32_t ds_full = bar(6);
-  const uint32_t acc_done = bar(7);
+  auto s_full = [&](int hh) { return bar(5 + hh); };
+  auto ds_full = [&](int hh) { return bar(7 + hh); };
+  const uint32_t acc_done = bar(9);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
   const uint32_t q_smem = sbase + L::kFixOff;
@@ -444,14 +497,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(kv_full(s), 1);
       mbar_init(kv_empty(s), 1);
+      mbar_init(s_full(s), 1);
+      mbar_init(ds_full(s), kBM);
     }
-    mbar_init(s_full, 1);
-    mbar_init(ds_full, kBM);
     mbar_init(acc_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -459,9 +512,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // TMEM: [0,128) S then dS (bf16 pairs in [0,64)); [128,256) dP; [256,256+D) dQ
+  // TMEM: [0,128) S then dS (warpgroup w's bf16 pairs in [64w, 64w+32));
+  // [128,256) dP; [256,256+D) dQ
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     if (lane == 0 && n_kt > 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
@@ -490,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(kv_full(s), (last >> 1) & 1, &no_abort, p.err, p.timeout_ns);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     const bool leader = elect_one();
     auto wait = [&](uint32_t br, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(br, parity, abort_flag, p.err, p.timeout_ns));
@@ -503,30 +557,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = wait(kv_full(s), (jt >> 1) & 1);
       if (!ok) break;
       tc_fence_after();
+      const uint64_t kd = smem_desc_sw128(k_smem(s), 16, 1024);
+      const uint64_t vd = smem_desc_sw128(v_smem(s), 16, 1024);
       if (leader) {
-        mma_rows_x_rows<D>(tmem + 0, q_desc, smem_desc_sw128(k_smem(s), 16, 1024));     // S
-        mma_rows_x_rows<D>(tmem + 128, do_desc, smem_desc_sw128(v_smem(s), 16, 1024));  // dP
-        tc_commit(s_full);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          mma_rows_x_half<D>(tmem + kHalfN * hh, q_desc, kd, kHalfN * hh);          // S
+          mma_rows_x_half<D>(tmem + 128 + kHalfN * hh, do_desc, vd, kHalfN * hh);   // dP
+          tc_commit(s_full(hh));
+        }
       }
-      ok = wait(ds_full, jt & 1);
+      const uint64_t k_mn = smem_desc_sw128(k_smem(s), L::kChunkBytes, 1024);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        ok = wait(ds_full(hh), jt & 1);
+        if (!ok) break;
+        tc_fence_after();
+        // dQ += dS K_j over this half's keys (K_j read MN-major: D contiguous)
+        if (leader)
+          mma_half_x_tile<D>(tmem + 256, tmem + kHalfN * hh, k_mn, kHalfN * hh, jt > 0 || hh > 0);
+      }
       if (!ok) break;
-      tc_fence_after();
-      if (leader) {
-        // dQ += dS K_j (K_j read MN-major: the head dimension is contiguous)
-        mma_tmem_x_tile<D>(tmem + 256, tmem + 0,
-                           smem_desc_sw128(k_smem(s), L::kChunkBytes, 1024), jt > 0);
-        tc_commit(kv_empty(s));
-      }
+      if (leader) tc_commit(kv_empty(s));
     }
     if (leader) tc_commit(acc_done);
     volatile int no_abort = 0;
     mbar_wait(acc_done, 0, &no_abort, p.err, p.timeout_ns);
   } else {
-    const int r = tid;
+    const int wg = warp >> 2;                           // keys 64 wg .. 64 wg + 63
+    const int r = (warp & 3) * 32 + lane;
     const int row = i * kBM + r;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_base;
-    const uint32_t tP = tmem + lane_base + 128;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + kHalfN * wg;
+    const uint32_t tP = tmem + lane_base + 128 + kHalfN * wg;
     const size_t grow = static_cast<size_t>(bh) * p.Nq + row;
     float lse2 = INFINITY, dl = 0.f;
     if (row < p.Nq) {
@@ -535,20 +598,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
     const uint64_t nl2 = f2_pack(-lse2, -lse2);
+    const uint64_t dl2 = f2_pack(dl, dl);
     bool ok = true;
     for (int jt = 0; ok && jt < n_kt; ++jt) {
-      const bool got = mbar_wait(s_full, jt & 1, abort_flag, p.err, p.timeout_ns);
+      const bool got = mbar_wait(s_full(wg), jt & 1, abort_flag, p.err, p.timeout_ns);
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int kbase = jt * kBM;
-      const bool need_mask = (kbase + kBM > p.Nk) || (p.causal && kbase + kBM - 1 > i * kBM + off);
+      const int kbase = jt * kBM + kHalfN * wg;        // first key of this half
+      const bool need_mask =
+          (kbase + kHalfN > p.Nk) || (p.causal && kbase + kHalfN - 1 > i * kBM + off);
       int lim = p.Nk - 1 - kbase;
       if (p.causal) lim = min(lim, row + off - kbase);
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t sv[32], dv[32];
         tmem_ld32(tS + 32 * c, sv, p.err);
         tmem_ld32(tP + 32 * c, dv, p.err);
@@ -564,30 +629,35 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (32 * c + e > lim) p0 = 0.f;
             if (32 * c + e + 1 > lim) p1 = 0.f;
           }
-          pk[e >> 1] = pack_bf16x2(p0 * (__uint_as_float(dv[e]) - dl),
-                                   p1 * (__uint_as_float(dv[e + 1]) - dl));
+          float d0, d1;
+          f2_unpack(f2_mul(f2_pack(p0, p1),
+                           f2_sub(f2_pack(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])),
+                                  dl2)),
+                    d0, d1);
+          pk[e >> 1] = pack_bf16x2(d0, d1);
         }
         tmem_st16(tS + 16 * c, pk, p.err);     // over columns already read
       }
       tmem_wait_st(p.err);
       tc_fence_before();
-      mbar_arrive(ds_full);
+      mbar_arrive(ds_full(wg));
     }
     const bool fin = ok && (n_kt == 0 || mbar_wait(acc_done, 0, abort_flag, p.err, p.timeout_ns));
     if (__all_sync(0xffffffffu, fin)) {
       tc_fence_after();
       uint16_t* dst = p.dq + grow * D;
+      const int c0 = wg * (D / 2);
       if (n_kt == 0) {
-        if (row < p.Nq) store_zero_row<D>(dst);
+        if (row < p.Nq) store_zero_cols(dst, c0, D / 2);
       } else {
-        store_row_bf16<D>(tmem + lane_base + 256, p.scale, dst, row < p.Nq, p.err);
+        store_cols_bf16(tmem + lane_base + 256, c0, D / 2, p.scale, dst, row < p.Nq, p.err);
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);

@@ -30,11 +30,13 @@
 // raw scores to scaled log2 units with the tile's factor
 // scale * log2(e) * q_scale * k_scale_j and writes P back over the first 32
 // columns of its S tile as E4M3 (four per column), offset so that the row's
-// reference maximum maps to 2^8: p = 2^(x - m_ref + 8).  With a lazy-rescale
-// threshold of 0.5 every p is at most 2^8.5 < 448, and entries down to 2^-14
-// of the maximum stay normal E4M3 numbers.  The row sum L is taken over the
-// unrounded p; O is multiplied by v_scale / L at the end and LSE removes the
-// offset.
+// reference maximum maps to 2^6: p = 2^(x - m_ref + 6).  With a lazy-rescale
+// threshold of 2.5 every p is at most 2^8.5 < 448 (the reference moves, and O is
+// rescaled, only when a tile's maximum exceeds it by more than 2.5), and entries
+// down to 2^-12 of the reference stay normal E4M3 numbers (below that the
+// subnormal spacing 2^-9 is at most 2^-15 of the row's largest p).  The row sum
+// L is taken over the unrounded p; O is multiplied by v_scale / L at the end
+// and LSE removes the offset.
 #include <algorithm>
 #include <cfloat>
 #include <cstdio>
@@ -96,34 +98,38 @@ __global__ void __launch_bounds__(kQuantThreads)
 #pragma unroll
     for (int e = 0; e < E; ++e) mult[e] = __fmul_rn(__ldg(signs + lane * E + e), c);
   }
+  // all 16 rows' loads are issued before any arithmetic, so they are in flight
+  // together (rows past N read as zero and are not stored)
+  uint32_t w[kQuantRowsPerWarp][E / 2];
+#pragma unroll
+  for (int i = 0; i < kQuantRowsPerWarp; ++i) {
+    const int row = row0 + i;                    // warp-uniform
+    const uint16_t* src = x + slice + static_cast<size_t>(row) * D + lane * E;
+    if constexpr (E == 4) {
+      uint2 u = make_uint2(0u, 0u);
+      if (row < N) u = __ldg(reinterpret_cast<const uint2*>(src));
+      w[i][0] = u.x;
+      w[i][1] = u.y;
+    } else {
+      w[i][0] = row < N ? __ldg(reinterpret_cast<const uint32_t*>(src)) : 0u;
+    }
+  }
   float v[kQuantRowsPerWarp][E];
   float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < kQuantRowsPerWarp; ++i) {
-    const int row = row0 + i;                    // warp-uniform
-    if (row < N) {
-      const uint16_t* src = x + slice + static_cast<size_t>(row) * D + lane * E;
-      uint32_t w[E / 2];
-      if constexpr (E == 4) {
-        const uint2 u = __ldg(reinterpret_cast<const uint2*>(src));
-        w[0] = u.x;
-        w[1] = u.y;
-      } else {
-        w[0] = __ldg(reinterpret_cast<const uint32_t*>(src));
-      }
 #pragma unroll
-      for (int e = 0; e < E / 2; ++e) {
-        v[i][2 * e] = __uint_as_float(w[e] << 16);
-        v[i][2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
-      }
-      if constexpr (ROT) {
-#pragma unroll
-        for (int e = 0; e < E; ++e) v[i][e] = __fmul_rn(v[i][e], mult[e]);
-        fwht_row<E>(v[i], lane);
-      }
-#pragma unroll
-      for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(v[i][e]));
+    for (int e = 0; e < E / 2; ++e) {
+      v[i][2 * e] = __uint_as_float(w[i][e] << 16);
+      v[i][2 * e + 1] = __uint_as_float(w[i][e] & 0xffff0000u);
     }
+    if constexpr (ROT) {
+#pragma unroll
+      for (int e = 0; e < E; ++e) v[i][e] = __fmul_rn(v[i][e], mult[e]);
+      fwht_row<E>(v[i], lane);
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(v[i][e]));
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
@@ -206,8 +212,9 @@ constexpr int kBN = 128;            // keys per tile
 constexpr int kD = 128;             // head dimension (one byte per element)
 constexpr int kTile = kBM * kD;     // bytes of a Q, K or V tile
 constexpr int kSlots = 10;          // K/V ring slots
-constexpr float kTau = 0.5f;        // lazy-rescale threshold (log2 units)
-constexpr float kPOff = 8.f;        // p = 2^(x - m_ref + kPOff)
+constexpr float kTau = 2.5f;        // lazy-rescale threshold (log2 units)
+constexpr float kPOff = 6.f;        // p = 2^(x - m_ref + kPOff)
+constexpr float kPScale = 64.f;     // 2^kPOff
 constexpr int kThreads = 384;
 #ifndef FA_FP8_HALF_EXP
 #define FA_FP8_HALF_EXP 0
@@ -215,7 +222,7 @@ constexpr int kThreads = 384;
 // 1: the exponentials of P in f16 pairs (ex2.approx.f16x2), converted straight
 // to E4M3; 0: one fp32 exponential per element.
 constexpr bool kHalfExp = FA_FP8_HALF_EXP != 0;
-constexpr uint32_t kF16x2Off = 0x5C005C00u;   // (256, 256) in f16: 2^kPOff
+constexpr uint32_t kF16x2Off = 0x54005400u;   // (64, 64) in f16: 2^kPOff
 constexpr uint32_t kRegsControl = 72;
 constexpr uint32_t kRegsSoftmax = 216;
 static_assert(kRegsControl * 128 + kRegsSoftmax * 256 <= 384 * 168, "register split");
@@ -627,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = false;
       } else {
         tc_fence_after();
-        const float l_p = kHalfExp ? l * 256.f : l;   // the sum of the p that P holds
+        const float l_p = kHalfExp ? l * kPScale : l;   // the sum of the p that P holds
         const float inv = l > 0.f ? v_s / l_p : 0.f;
 #pragma unroll 1
         for (int cc = 0; cc < kD / 32; ++cc) {
