@@ -24,7 +24,7 @@
 // (setmaxnreg): 72 and 216 per-thread registers over 128 + 256 threads equal
 // the 384 x 168 the block is launched with.
 // Tensor memory (512 columns x 128 lanes, fp32):
-//   [  0,128) S0 = Q0 K^T  (its first 64 columns are reused for P0 as bf16 pairs)
+//   [  0,128) S0 = Q0 K^T  (its last 64 columns are reused for P0 as bf16 pairs)
 //   [128,256) S1 = Q1 K^T  (P1 likewise)
 //   [256,256+D) O0,  [256+D,256+2D) O1  -- the running unnormalised outputs
 // Per key tile j the MMA thread issues, in order: PV0_j, S0_{j+1}, PV1_j, S1_{j+1},
@@ -57,6 +57,22 @@ constexpr float kTau = 8.0f;   // lazy-rescale threshold (log2 units)
 #endif
 // Of every 16 column pairs, this many use the FMA-pipe exp2 (the rest use MUFU).
 constexpr int kPolyPairs = FA_POLY_PAIRS;
+#ifndef FA_S_SPLIT
+#define FA_S_SPLIT 1
+#endif
+// At D = 64: the keys 0-63 of S_{j+1} are computed once the first half of P_j
+// is out (the softmax read all of S_j before writing it, and P_j only occupies
+// columns 64-127), so only the other half of S_{j+1} remains between the
+// release of P_j's second half and the next softmax (D = 64 is bound by that chain:
+// 0.1219 vs 0.1259 ms on the (2, 8, 4096, 64) workload).  At D = 128 the two
+// N = 64 products read Q from shared memory twice, and the S products are
+// already at the shared-memory bandwidth limit: measured 8 % slower there.
+template <int D>
+constexpr bool split_s() { return FA_S_SPLIT != 0 && D == 64; }
+#ifndef FA_MAX_CHAINS
+#define FA_MAX_CHAINS 4
+#endif
+constexpr int kMaxChains = FA_MAX_CHAINS;   // independent chains of the row maximum
 constexpr int kThreads = 384;
 constexpr uint32_t kRegsControl = 72;    // warps 8-11
 constexpr uint32_t kRegsSoftmax = 216;   // warps 0-7
@@ -412,7 +428,83 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ------------------------------------------------------------ TMA producer
       // Items in order; per item both Q tiles (a tile past Nq reads as zeros),
       // then K_j, V_j through the ring, whose position runs on across items.
-      if (lane == 0) {
+      if constexpr (MODE == kPaged) {
+        // A key tile is eight 16-token pages: the whole warp walks the items and
+        // waits (warp-uniform), lane 0 posts each tile's bytes, and lane
+        // pg * kChunks + ch reads page pg's block-table entry and issues its
+        // chunk ch box, so the 8 (or 16) boxes and table reads leave together.
+        // Keys past the sequence read its first page (masked later, but finite);
+        // an id outside the pool is flagged and replaced by page 0.
+        if (lane == 0) {
+          tma_prefetch_desc(&tmQ);
+          tma_prefetch_desc(&tmK);
+          tma_prefetch_desc(&tmV);
+        }
+        auto wait_all = [&](uint32_t br, uint32_t parity) {
+          return __all_sync(0xffffffffu, mbar_wait(br, parity, abort_flag, p.err, p.timeout_ns));
+        };
+        constexpr int kBoxes = (kBN / kPageTok) * L::kChunks;
+        const int pg = lane / L::kChunks, ch = lane % L::kChunks;
+        int pos = 0, items = 0;
+        bool ok = true;
+        ItemWalker<MODE> walk;
+        walk.init(p, cta, C, sorted, n_sorted);
+        FwdItem it;
+        while (ok && walk.next(p, it)) {
+          const int n_max = max(it.n0, it.n1);
+          if (n_max == 0) continue;
+          if (items > 0 && !wait_all(q_empty, (items - 1) & 1)) break;
+          if (lane == 0) {
+            for (int t = 0; t < 2; ++t) {
+              mbar_arrive_expect_tx(q_full(t), L::kTileBytes);
+              const uint32_t dst = sbase + L::kQOff + t * L::kTileBytes;
+              for (int c2 = 0; c2 < L::kChunks; ++c2)   // [total_q, Hq, D]: box {64, 1, 128}
+                tma_load_3d(dst + c2 * L::kChunkBytes, &tmQ, q_full(t), c2 * 64, it.h,
+                            it.q_start + it.q_row0 + t * kBM);
+            }
+          }
+          ++items;
+          const int* tab = p.block_table + static_cast<size_t>(it.b) * p.max_pages;
+          for (int j = 0; j < n_max && ok; ++j) {
+            // this lane's page of key tile j, shared by its K and V boxes
+            int page = 0;
+            if (lane < kBoxes) {
+              const int tok = j * kBN + pg * kPageTok;
+              page = __ldg(tab + (tok < it.nk ? tok / kPageTok : 0));
+              if (page < 0 || page >= p.num_pages) {
+                atomicOr(p.err, kErrBadIndex);
+                page = 0;
+              }
+            }
+            for (int w = 0; w < 2; ++w, ++pos) {
+              const int slot = pos % L::kSlots;
+              const uint32_t ph = (pos / L::kSlots) & 1;
+              if (!wait_all(kv_empty(slot), ph ^ 1)) {
+                ok = false;
+                break;
+              }
+              if (lane == 0) mbar_arrive_expect_tx(kv_full(slot), L::kTileBytes);
+              __syncwarp();
+              const uint32_t dst = sbase + L::kKVOff + slot * L::kTileBytes;
+              const void* tm = w ? static_cast<const void*>(&tmV) : static_cast<const void*>(&tmK);
+              if (lane < kBoxes)
+                tma_load_3d(dst + ch * L::kChunkBytes + pg * kPageTok * 128, tm, kv_full(slot),
+                            ch * 64, it.hkv, page * kPageTok);
+            }
+          }
+        }
+        // Every issued copy must land before the CTA may exit (also on abort).
+        if (lane == 0) {
+          volatile int no_abort = 0;
+          if (items > 0)
+            for (int t = 0; t < 2; ++t)
+              mbar_wait(q_full(t), (items - 1) & 1, &no_abort, p.err, p.timeout_ns);
+          for (int sl = 0; sl < L::kSlots && sl < pos; ++sl) {
+            const int last = sl + ((pos - 1 - sl) / L::kSlots) * L::kSlots;
+            mbar_wait(kv_full(sl), (last / L::kSlots) & 1, &no_abort, p.err, p.timeout_ns);
+          }
+        }
+      } else if (lane == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
@@ -451,31 +543,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               mbar_arrive_expect_tx(kv_full(slot), L::kTileBytes);
               const uint32_t dst = sbase + L::kKVOff + slot * L::kTileBytes;
               const void* tm = w ? static_cast<const void*>(&tmV) : static_cast<const void*>(&tmK);
-              if constexpr (MODE == kPaged) {
-                // eight 16-token boxes, one per page; keys past the sequence read its
-                // first page (masked later, but finite); an id outside the pool is
-                // flagged and replaced by page 0
-                const int* tab = p.block_table + static_cast<size_t>(it.b) * p.max_pages;
-                for (int pg = 0; pg < kBN / kPageTok; ++pg) {
-                  const int tok = j * kBN + pg * kPageTok;
-                  int page = __ldg(tab + (tok < it.nk ? tok / kPageTok : 0));
-                  if (page < 0 || page >= p.num_pages) {
-                    atomicOr(p.err, kErrBadIndex);
-                    page = 0;
-                  }
-                  for (int ch = 0; ch < L::kChunks; ++ch)
-                    tma_load_3d(dst + ch * L::kChunkBytes + pg * kPageTok * 128, tm,
-                                kv_full(slot), ch * 64, it.hkv, page * kPageTok);
-                }
-              } else {
-                for (int ch = 0; ch < L::kChunks; ++ch) {
-                  if (RAGGED)
-                    tma_load_3d(dst + ch * L::kChunkBytes, tm, kv_full(slot), ch * 64, it.hkv,
-                                it.k_start + j * kBN);
-                  else
-                    tma_load_3d(dst + ch * L::kChunkBytes, tm, kv_full(slot), ch * 64,
-                                j * kBN, kv_z);
-                }
+              for (int ch = 0; ch < L::kChunks; ++ch) {
+                if (RAGGED)
+                  tma_load_3d(dst + ch * L::kChunkBytes, tm, kv_full(slot), ch * 64, it.hkv,
+                              it.k_start + j * kBN);
+                else
+                  tma_load_3d(dst + ch * L::kChunkBytes, tm, kv_full(slot), ch * 64,
+                              j * kBN, kv_z);
               }
             }
           }
@@ -527,12 +601,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_commit(s_full(t));
           }
         };
+        // Keys [key0, key0 + 64) of S_t = Q_t K^T into its columns key0 ..: the
+        // K rows start key0 * 128 bytes into each swizzle-atom column (a whole
+        // number of 8-row atoms); the second call commits S_t as complete.
+        constexpr uint32_t idesc_s64 = idesc_f16(kBM, kBN / 2, BF16, false);
+        auto issue_s_keys = [&](int t, int slot, int key0, bool last) {
+          const uint64_t a0 = t ? desc_q1 : desc_q0;
+          const uint64_t b0 =
+              desc_k + static_cast<uint64_t>((slot * L::kTileBytes + key0 * 128) >> 4);
+          const uint32_t d = tmem + t * 128 + key0;
+          if (leader) {
+  #pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t off =
+                  static_cast<uint64_t>(((kk >> 2) * L::kChunkBytes + (kk & 3) * 32) >> 4);
+              mma_ss(d, a0 + off, b0 + off, idesc_s64, kk > 0 ? 1u : 0u);
+            }
+            if (last) tc_commit(s_full(t));
+          }
+        };
         // O_t += P_t V over keys [64 h, 64 h + 64): A = P from TMEM (bf16 pairs),
         // B = V tile, MN-major (D contiguous)
         auto issue_pv_half = [&](int t, int slot, int h, bool accumulate) {
           const uint64_t b0 = desc_v + static_cast<uint64_t>((slot * L::kTileBytes) >> 4);
           const uint32_t d = tmem + 256 + t * D;
-          const uint32_t a = tmem + t * 128;
+          const uint32_t a = tmem + t * 128 + 64;   // P: 16-bit pairs in S's columns 64-127
           if (leader) {
   #pragma unroll
             for (int k4 = 0; k4 < kBN / 32; ++k4) {
@@ -576,18 +669,35 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!ok) continue;
               tc_fence_after();
               issue_pv_half(t, slot_of(vpos), 0, j > 0);
+              if constexpr (split_s<D>()) {
+                // P_t(j)'s first half is out, so the softmax has read all of S_t(j):
+                // keys 0-63 of S_t(j + 1) go into columns P_t(j) does not use
+                if (j + 1 < nt) {
+                  if (!k_ready) {
+                    ok = wait(kv_full(slot_of(kpos)), phase_of(kpos));
+                    k_ready = true;
+                    if (!ok) continue;
+                    tc_fence_after();
+                  }
+                  issue_s_keys(t, slot_of(kpos), 0, false);
+                }
+              }
               ok = wait(p_half(t, 1), par);
               if (!ok) continue;
               tc_fence_after();
               issue_pv_half(t, slot_of(vpos), 1, true);
               if (j + 1 < nt) {
-                if (!k_ready) {
-                  ok = wait(kv_full(slot_of(kpos)), phase_of(kpos));
-                  k_ready = true;
-                  if (!ok) continue;
-                  tc_fence_after();
+                if constexpr (split_s<D>()) {
+                  issue_s_keys(t, slot_of(kpos), kBN / 2, true);   // after P V has read P_t(j)
+                } else {
+                  if (!k_ready) {
+                    ok = wait(kv_full(slot_of(kpos)), phase_of(kpos));
+                    k_ready = true;
+                    if (!ok) continue;
+                    tc_fence_after();
+                  }
+                  issue_s(t, slot_of(kpos));
                 }
-                issue_s(t, slot_of(kpos));
               } else {
                 commit(o_full(t));
               }
@@ -614,6 +724,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = tid & 127;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + t * 128;
+    const uint32_t tP = tS + 64;             // P as 16-bit pairs over S's keys 64-127
     const uint32_t tO = tmem + lane_base + 256 + t * D;
     int tiles = 0, outs = 0;     // S tiles and O tiles of this slot in earlier items (phases)
     bool ok = true;
@@ -669,19 +780,44 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 128; ++e)
             if (e > lim) s[e] = __float_as_uint(-INFINITY);
         }
-        // row maximum: 8 independent three-input-max chains, then a short tree
-        float acc[8];
+        const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
+        uint64_t sum2[4] = {0, 0, 0, 0};   // four independent packed partial sums
+        // exponentials of the 32 columns 32 c .. 32 c + 31 against reference -nm,
+        // packed to 16-bit pairs (unmasked tiles may put the first kPolyPairs
+        // pairs of every 32 columns on the FMA pipe)
+        auto exp_cols = [&](int c, float nm, uint32_t (&pk)[16]) {
+          const uint64_t nm2 = f2_pack(nm, nm);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) acc[k] = __uint_as_float(s[k]);
+          for (int e = 0; e < 16; ++e) {
+            float x0, x1, p0, p1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(s[32 * c + 2 * e]),
+                                     __uint_as_float(s[32 * c + 2 * e + 1])), c2, nm2), x0, x1);
+            if (!need_mask && e < kPolyPairs) {
+              exp2_fma_pair(x0, x1, p0, p1);
+            } else {
+              p0 = ex2(x0);
+              p1 = ex2(x1);
+            }
+            sum2[e & 3] = f2_add(sum2[e & 3], f2_pack(p0, p1));
+            pk[e] = BF16 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
+          }
+        };
+        // row maximum: kMaxChains independent three-input-max chains, then a short tree
+        float acc[kMaxChains];
 #pragma unroll
-        for (int e = 8; e + 16 <= 128; e += 16)
+        for (int k = 0; k < kMaxChains; ++k) acc[k] = __uint_as_float(s[k]);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            acc[k] = fmax3(acc[k], __uint_as_float(s[e + k]), __uint_as_float(s[e + 8 + k]));
+        for (int e = kMaxChains; e + 2 * kMaxChains <= 128; e += 2 * kMaxChains)
 #pragma unroll
-        for (int k = 0; k < 8; ++k) acc[k] = fmaxf(acc[k], __uint_as_float(s[120 + k]));
-        const float mx = fmax3(fmax3(acc[0], acc[1], acc[2]), fmax3(acc[3], acc[4], acc[5]),
-                               fmaxf(acc[6], acc[7]));
+          for (int k = 0; k < kMaxChains; ++k)
+            acc[k] = fmax3(acc[k], __uint_as_float(s[e + k]),
+                           __uint_as_float(s[e + kMaxChains + k]));
+#pragma unroll
+        for (int k = 0; k < kMaxChains; ++k)
+          acc[k] = fmaxf(acc[k], __uint_as_float(s[128 - kMaxChains + k]));
+#pragma unroll
+        for (int k = 1; k < kMaxChains; ++k) acc[0] = fmaxf(acc[0], acc[k]);
+        const float mx = acc[0];
         const float m_tile = mx * p.scale_log2;
         const bool move = m_tile > m_used + kTau;
         float alpha = 1.f;
@@ -704,57 +840,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
-        const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
-        const uint64_t nm2 = f2_pack(neg_m, neg_m);
-        uint64_t sum2[4] = {0, 0, 0, 0};   // four independent packed partial sums
-        if (need_mask) {
-          // masked tiles: every exponential on MUFU (exactly 0 for masked scores)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t pk[16];
+        for (int c = 0; c < 2; ++c) {
+          uint32_t pk[16];
+          exp_cols(c, neg_m, pk);
+          tmem_st16(tP + 16 * c, pk, p.err);
+        }
+        tmem_wait_st(p.err);                 // keys 0-63 of P are in place
+        tc_fence_before();
+        mbar_arrive(p_half(t, 0));
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float x0, x1;
-              f2_unpack(f2_fma(f2_pack(__uint_as_float(s[32 * c + 2 * e]),
-                                       __uint_as_float(s[32 * c + 2 * e + 1])), c2, nm2), x0, x1);
-              const float p0 = ex2(x0), p1 = ex2(x1);
-              sum2[e & 3] = f2_add(sum2[e & 3], f2_pack(p0, p1));
-              pk[e] = BF16 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
-            }
-            tmem_st16(tS + 16 * c, pk, p.err);
-            if (c == 1) {                        // keys 0-63 of P are in place
-              tmem_wait_st(p.err);
-              tc_fence_before();
-              mbar_arrive(p_half(t, 0));
-            }
-          }
-        } else {
-          // unmasked tiles: the first kPolyPairs pairs of every 32 columns on the
-          // FMA pipe, the rest on MUFU, so both units share the exponentials
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float x0, x1, p0, p1;
-              f2_unpack(f2_fma(f2_pack(__uint_as_float(s[32 * c + 2 * e]),
-                                       __uint_as_float(s[32 * c + 2 * e + 1])), c2, nm2), x0, x1);
-              if (e < kPolyPairs) {
-                exp2_fma_pair(x0, x1, p0, p1);
-              } else {
-                p0 = ex2(x0);
-                p1 = ex2(x1);
-              }
-              sum2[e & 3] = f2_add(sum2[e & 3], f2_pack(p0, p1));
-              pk[e] = BF16 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
-            }
-            tmem_st16(tS + 16 * c, pk, p.err);
-            if (c == 1) {                        // keys 0-63 of P are in place
-              tmem_wait_st(p.err);
-              tc_fence_before();
-              mbar_arrive(p_half(t, 0));
-            }
-          }
+        for (int c = 2; c < 4; ++c) {
+          uint32_t pk[16];
+          exp_cols(c, neg_m, pk);
+          tmem_st16(tP + 16 * c, pk, p.err);
         }
         float sa, sb;
         f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), sa, sb);

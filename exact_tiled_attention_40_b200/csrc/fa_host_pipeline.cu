@@ -1,9 +1,10 @@
 // Forward from host buffers: fa_fwd with the inputs in host memory and the
 // outputs wanted back there.
 //
-// The work is cut into about eight chunks of whole sequences, or of whole GQA
-// groups of one sequence when there are fewer than eight sequences; each chunk
-// is contiguous in every tensor.  Chunk c's inputs are copied in on a copy
+// The work is cut into chunks of whole sequences (B >= 8), of whole GQA groups
+// of the one sequence (B = 1), both in the proportions 1:3:3:1, or of about
+// 8 / B group ranges per sequence otherwise; each chunk is contiguous in every
+// tensor.  Chunk c's inputs are copied in on a copy
 // stream while chunk c - 1 is computed on the caller's stream and chunk c - 2's
 // outputs are copied out on a second copy stream, so the host-to-device and
 // device-to-host transfers (separate directions of the link) overlap each
@@ -49,13 +50,34 @@ struct Chunk {
   int g0, ng;   // KV-head groups of each (all of them when nb > 1)
 };
 
+// Sizes of the chunks of n units in the proportions 1:3:3:1: a small first
+// chunk lets the kernels start early and a small last chunk leaves little to
+// copy out after the last kernel, while the middle chunks keep both copy
+// directions busy (B1 Hq32 Hkv8 N8192 D128 causal prefill on a B200: 2.69 ms
+// per call against 2.87 ms with eight equal chunks and 2.76 ms with four).
+std::vector<int> chunk_sizes(int n) {
+  if (n < 4) return std::vector<int>(n, 1);
+  const int edge = std::max(1, n / 8);
+  const int mid = n - 2 * edge;
+  return {edge, (mid + 1) / 2, mid / 2, edge};
+}
+
 std::vector<Chunk> plan_chunks(int B, int Hkv) {
-  constexpr int kTarget = 8;
   std::vector<Chunk> out;
-  if (B >= kTarget) {
-    const int per = (B + kTarget - 1) / kTarget;
-    for (int b0 = 0; b0 < B; b0 += per) out.push_back({b0, std::min(per, B - b0), 0, Hkv});
-  } else {
+  if (B >= 8) {                       // chunks of whole sequences
+    int b0 = 0;
+    for (int n : chunk_sizes(B)) {
+      out.push_back({b0, n, 0, Hkv});
+      b0 += n;
+    }
+  } else if (B == 1) {                // chunks of whole GQA groups of the sequence
+    int g0 = 0;
+    for (int n : chunk_sizes(Hkv)) {
+      out.push_back({0, 1, g0, n});
+      g0 += n;
+    }
+  } else {                            // each sequence in about 8 / B group chunks
+    constexpr int kTarget = 8;
     const int parts = std::min(Hkv, (kTarget + B - 1) / B);
     const int per = (Hkv + parts - 1) / parts;
     for (int b = 0; b < B; ++b)

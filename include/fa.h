@@ -145,8 +145,9 @@ int fa_fwd_paged(const void* q, const void* kcache, const void* vcache,
  *   q_dev, k_dev, v_dev, o_dev, lse_dev: device buffers of the same sizes, owned
  *     by the caller, used as staging (their contents are overwritten)
  *   lse_host and lse_dev are both given or both NULL.
- * The work is cut into about eight chunks (whole sequences, or whole GQA groups
- * of a sequence); each chunk's inputs are copied in while the previous chunk is
+ * The work is cut into chunks of whole sequences (B >= 8) or whole GQA groups
+ * of a sequence (sized 1:3:3:1 when B >= 8 or B = 1: small first and last
+ * chunks); each chunk's inputs are copied in while the previous chunk is
  * computed and the one before it copied out, on two library-owned copy streams
  * ordered against `stream` by events: the call is asynchronous on `stream` like
  * fa_fwd, and the host outputs are complete once `stream` reaches the point of
