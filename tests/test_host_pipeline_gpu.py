@@ -17,6 +17,7 @@ CASES = [
     PrefillCase("host_groups", 1, 32, 8, 1024, 1024, 128, seed=100, causal=True),
     PrefillCase("host_three_seqs", 3, 8, 8, 300, 300, 64, seed=101),
     PrefillCase("host_many_seqs", 11, 4, 2, 260, 400, 128, seed=102, causal=True),
+    PrefillCase("host_two_groups", 1, 4, 2, 333, 333, 64, seed=103, causal=True),
 ]
 
 
