@@ -457,13 +457,19 @@ def dense_prefill_rows(fa, dev, stream, flush, warmup, steps, peaks, peak_src):
             ms = statistics.median(ts)
             tf = c.flops / (ms * 1e-3) / 1e12
             otf, odt, sample = sample_fn(c)
+            # a launch of a tenth of a second or more runs under the power cap:
+            # the GEMM peak measured over seconds is its denominator
+            sustained = ms >= 100.0
+            peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+            kind = "sustained" if sustained else "burst"
             out[key] = {"workload": c.name, "dtype": c.dtype, "value": tf, "unit": "TFLOP/s",
                         "ms_per_launch": ms, "launches_timed": n_steps,
                         "roofline": {"bound": "tensor", "achieved": tf,
-                                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                                     "frac": tf / peaks["bf16_tflops"],
-                                     "peak_source": f"{peak_src} burst bf16 (fp16 dense "
+                                     "peak": peak, "unit": "TFLOP/s",
+                                     "frac": tf / peak,
+                                     "peak_source": f"{peak_src} {kind} bf16 (fp16 dense "
                                                     "tensor peak is the same)",
+                                     "frac_of_burst": tf / peaks["bf16_tflops"],
                                      "frac_of_nominal_2250": tf / 2250.0},
                         "cpu_baseline": {"value": otf, "unit": "TFLOP/s",
                                          "cores": cpu_threads(), "kind": "oracle",
