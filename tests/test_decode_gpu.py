@@ -54,6 +54,14 @@ def test_fewer_cache_chunks_than_sms(cuda_device):
     check(case, *make_decode(case))
 
 
+def test_many_sequences_offsets_in_global_memory(cuda_device):
+    """5000 short sequences: more than the 4096 whose half-page offsets the
+    stream kernel's producer keeps in shared memory, so it searches them in
+    global memory, and the merge runs 5000 blocks."""
+    case = DecodeCase("many", 5000, 8, 2, 128, 16, 1, 40, 16000, seed=53)
+    check(case, *make_decode(case))
+
+
 def test_zero_length_sequence(cuda_device):
     case = DecodeCase("zero", 3, 8, 2, 128, 16, 5, 40, 20, seed=50)
     q, kc, vc, table, lens = make_decode(case)

@@ -49,6 +49,13 @@ def test_full_prompt_non_causal(cuda_device):
                            nq=(50, 260, 3), nk=(50, 260, 1100)))
 
 
+def test_more_sequences_than_the_sorted_list_holds(cuda_device):
+    """1100 sequences (past the 1024 the kernel sorts) of up to 100 cached
+    keys, each querying all of them."""
+    check(PagedPrefillCase("many", 1100, 4, 2, 128, True, seed=114, num_pages=8000, lo=1,
+                           hi=100))
+
+
 def test_head_dim_64(cuda_device):
     check(PagedPrefillCase("d64", 5, 8, 2, 64, True, seed=112, num_pages=500, lo=1, hi=900))
 

@@ -58,6 +58,12 @@ def test_sequence_without_keys_non_causal(cuda_device):
     assert torch.all(o[200:205] == 0)
 
 
+def test_more_sequences_than_the_sorted_list_holds(cuda_device):
+    """1500 short sequences: past the 1024 whose work the kernel sorts in
+    shared memory, so the CTAs walk the (pair, sequence) items in plain order."""
+    check(VarlenCase("many", 1500, 4, 2, 64, "bf16", True, seed=96, lo=1, hi=300))
+
+
 def test_mha_fp16_d64(cuda_device):
     check(VarlenCase("fp16", 5, 8, 8, 64, "fp16", True, seed=93, lo=1, hi=700))
 
