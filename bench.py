@@ -99,14 +99,19 @@ def recorded_traffic(kernel: str, source: str):
 
 
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """Samples SM clocks and throttle reasons with nvidia-smi every 20 ms while
+    running; the summary keeps the samples taken inside the timed region
+    (mark() brackets it), or all of them when none fell inside (a region shorter
+    than the sampling interval), and says which."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    INTERVAL_MS = 20
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
+        self.window = None
         out_dir = os.environ.get("FA_BENCH_OUT", os.path.join(ROOT, "bench_out"))
         self.path = os.path.join(out_dir, f"clocks_rank{index}.csv")
 
@@ -116,7 +121,7 @@ class ClockSampler:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.INTERVAL_MS)],
                 stdout=self.f, stderr=subprocess.DEVNULL)
             time.sleep(0.3)
         except Exception:
@@ -132,28 +137,40 @@ class ClockSampler:
                 self.proc.kill()
             self.f.close()
 
+    def mark(self, start: float, end: float):
+        """The timed region in wall-clock seconds (time.time())."""
+        self.window = (start, end)
+
+    @staticmethod
+    def parse(lines, window=None):
+        """Summary of nvidia-smi CSV lines (FIELDS order); `window` = (start, end)
+        in seconds since the epoch selects the samples taken inside it."""
+        import datetime
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        rows = []
+        for line in lines:
+            cols = [c.strip() for c in line.split(",")]
+            if len(cols) < 9:
+                continue
+            try:
+                ts = datetime.datetime.strptime(cols[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(cols[1]), float(cols[2]),
+                             [n for n, c in zip(names, cols[5:9]) if c.lower().startswith("active")]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        inside = [r for r in rows if window and window[0] <= r[0] <= window[1]]
+        used, where = (inside, "timed region") if inside else (rows, "whole run")
+        return {"sm_mhz": statistics.median(r[1] for r in used), "sm_max_mhz": used[-1][2],
+                "reasons": sorted({n for r in used for n in r[3]}), "samples": len(used),
+                "window": where, "interval_ms": ClockSampler.INTERVAL_MS}
+
     def summary(self):
         if self.proc is None or not os.path.exists(self.path):
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            cols = [c.strip() for c in line.split(",")]
-            if len(cols) < 8:
-                continue
-            try:
-                sm.append(float(cols[0]))
-                smax = float(cols[1])
-            except ValueError:
-                continue
-            for n, c in zip(names, cols[4:8]):
-                if c.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": ["no samples"]}
-        loaded = sorted(sm)[len(sm) // 4:] or sm       # drop the idle ramp-up samples
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        with open(self.path) as f:
+            return self.parse(f, self.window)
 
 
 def cpu_threads():
@@ -592,11 +609,13 @@ def main():
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         barrier()
+        w0 = time.time()
         t0.record(stream)
         for i in range(args.warmup, args.warmup + args.steps):
             step(i)
         t1.record(stream)
         barrier()
+        sampler.mark(w0, time.time())
     assert fa.device_status() == 0, fa.last_error()
     total_ms = t0.elapsed_time(t1)
     pre_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.warmup, args.warmup + args.steps)]
