@@ -78,6 +78,36 @@ __device__ __forceinline__ void fwht_row(float (&v)[E], int lane) {
     }
 }
 
+// The same transform with a row held by a lane pair, 64 consecutive elements
+// per lane (lane 2k + h holds 64 h .. 64 h + 63 of its row): the stages of
+// strides 1 to 32 stay in registers and only the stride-64 stage crosses
+// lanes.  The stages run in the same order with the same additions as
+// fwht_row, so every result is bit-identical.
+__device__ __forceinline__ void fwht_row_pair(float (&v)[64], int lane) {
+#pragma unroll
+  for (int h = 1; h < 64; h <<= 1)
+#pragma unroll
+    for (int e = 0; e < 64; ++e)
+      if (!(e & h)) {
+        const float a = v[e], c = v[e | h];
+        v[e] = __fadd_rn(a, c);
+        v[e | h] = __fsub_rn(a, c);
+      }
+#pragma unroll
+  for (int e = 0; e < 64; ++e) {
+    const float other = __shfl_xor_sync(0xffffffffu, v[e], 1);
+    v[e] = (lane & 1) ? __fsub_rn(other, v[e]) : __fadd_rn(v[e], other);
+  }
+}
+
+// Byte offset of 16-byte chunk `c` (0-15) of row `r` in a warp's staging area
+// of 16 rows x 256 bytes: chunks XOR-swizzled by the row within each 128-byte
+// half, so a lane pair per row reads and writes without bank conflicts beyond
+// the four wavefronts a 512-byte access needs.
+__device__ __forceinline__ uint32_t qstage_off(int r, int c) {
+  return static_cast<uint32_t>(r * 256 + (c & 8) * 16 + (((c & 7) ^ (r & 7)) << 4));
+}
+
 template <int D, bool ROT, int MODE>
 __global__ void __launch_bounds__(kQuantThreads)
     fa_quant_kernel(const uint16_t* __restrict__ x, uint8_t* __restrict__ codes,
@@ -85,6 +115,106 @@ __global__ void __launch_bounds__(kQuantThreads)
                     int groups) {
   constexpr int E = D / 32;
   __shared__ float warp_amax[kQuantThreads / 32];
+  if constexpr (D == 128) {
+    // Each warp's 16 rows (4 KB of bf16, contiguous in global memory) pass
+    // through shared memory: coalesced 16-byte global loads and stores, and a
+    // lane pair per row in registers.
+    __shared__ __align__(16) uint8_t stage_all[kQuantThreads / 32][16 * 256];
+    __shared__ float mult_sm[128];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int half = lane & 1;
+    const int rw = lane >> 1;                    // this lane's row within the warp's 16
+    const int g = blockIdx.x;
+    const int z = blockIdx.y;
+    const size_t slice = static_cast<size_t>(z) * N * D;
+    const int wrow0 = g * kQuantRows + warp * kQuantRowsPerWarp;
+    const uint32_t stage = smem_u32(stage_all[warp]);
+    if constexpr (ROT) {
+      if (threadIdx.x < 128)
+        mult_sm[threadIdx.x] = __fmul_rn(__ldg(signs + threadIdx.x), 0.0883883476483184405f);
+    }
+    // global -> shared: instruction k moves 512 contiguous bytes (rows 2k, 2k + 1)
+    const uint4* gsrc = reinterpret_cast<const uint4*>(x + slice + static_cast<size_t>(wrow0) * D);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int ci = k * 32 + lane;              // 16-byte chunk of the warp's 4 KB
+      const int r = ci >> 4;
+      const uint4 u = (wrow0 + r < N) ? __ldg(gsrc + ci) : make_uint4(0u, 0u, 0u, 0u);
+      st_shared_v4(stage + qstage_off(r, ci & 15), u.x, u.y, u.z, u.w);
+    }
+    __syncwarp();
+    float v[64];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      uint32_t u[4];
+      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3])
+                   : "r"(stage + qstage_off(rw, half * 8 + k)));
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        v[8 * k + 2 * q] = __uint_as_float(u[q] << 16);
+        v[8 * k + 2 * q + 1] = __uint_as_float(u[q] & 0xffff0000u);
+      }
+    }
+    if constexpr (ROT) {
+      __syncthreads();                           // mult_sm is written
+#pragma unroll
+      for (int e = 0; e < 64; ++e) v[e] = __fmul_rn(v[e], mult_sm[half * 64 + e]);
+      fwht_row_pair(v, lane);
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int e = 0; e < 64; ++e) amax = fmaxf(amax, fabsf(v[e]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if (lane == 0) warp_amax[warp] = amax;
+    __syncthreads();
+    amax = warp_amax[0];
+#pragma unroll
+    for (int w2 = 1; w2 < kQuantThreads / 32; ++w2) amax = fmaxf(amax, warp_amax[w2]);
+    if constexpr (MODE == kQuantSliceAmax) {
+      if (threadIdx.x == 0)
+        atomicMax(reinterpret_cast<unsigned int*>(scales) + z, __float_as_uint(amax));
+      return;
+    } else {
+      if constexpr (MODE == kQuantSlice)
+        amax = __uint_as_float(*reinterpret_cast<const volatile unsigned int*>(scales + z));
+      const float rr = amax > 0.f ? __fdiv_rn(448.f, amax) : 1.f;
+      if (MODE == kQuantGroups && threadIdx.x == 0)
+        scales[static_cast<size_t>(z) * groups + g] = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+      // codes -> shared (row rw's 128 code bytes at rw * 128, swizzled like the
+      // input's halves), then shared -> global, 512 contiguous bytes per instruction
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        uint32_t c4[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int e = 16 * k + 4 * q;
+          c4[q] = pack_e4m3x4(__fmul_rn(v[e], rr), __fmul_rn(v[e + 1], rr),
+                              __fmul_rn(v[e + 2], rr), __fmul_rn(v[e + 3], rr));
+        }
+        const int cc = half * 4 + k;             // 16-byte chunk of the 128-byte code row
+        st_shared_v4(stage + static_cast<uint32_t>(rw * 128 + ((cc ^ (rw & 7)) << 4)), c4[0],
+                     c4[1], c4[2], c4[3]);
+      }
+      __syncwarp();
+      uint4* gdst = reinterpret_cast<uint4*>(codes + slice + static_cast<size_t>(wrow0) * D);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int ci = k * 32 + lane;            // 16-byte chunk of the warp's 2 KB of codes
+        const int r = ci >> 3;
+        if (wrow0 + r < N) {
+          uint32_t u[4];
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3])
+                       : "r"(stage + static_cast<uint32_t>(r * 128 + (((ci & 7) ^ (r & 7)) << 4))));
+          gdst[ci] = make_uint4(u[0], u[1], u[2], u[3]);
+        }
+      }
+    }
+    return;
+  }
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int g = blockIdx.x;
