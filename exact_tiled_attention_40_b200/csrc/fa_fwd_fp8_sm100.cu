@@ -109,7 +109,7 @@ __device__ __forceinline__ uint32_t qstage_off(int r, int c) {
 }
 
 template <int D, bool ROT, int MODE>
-__global__ void __launch_bounds__(kQuantThreads)
+__global__ void __launch_bounds__(kQuantThreads, 3)
     fa_quant_kernel(const uint16_t* __restrict__ x, uint8_t* __restrict__ codes,
                     float* __restrict__ scales, const float* __restrict__ signs, int N,
                     int groups) {
