@@ -421,7 +421,6 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   __shared__ StageMeta meta[kMaxStages];
   __shared__ int abort_sm;
 
-  pdl_launch_dependents();   // the merge kernel may launch now; it waits for this grid
   const int c = blockIdx.x;
   const int C = gridDim.x;
   const int warp = threadIdx.x >> 5;
@@ -444,6 +443,9 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   }
   // Everything above overlaps the scan kernel; the half-page offsets are its output.
   pdl_wait();
+  // The merge kernel may launch once every CTA is past this point, so its launch
+  // implies that the scan has finished: it reads the offsets before its own wait.
+  pdl_launch_dependents();
   const int H = p.hb[p.B];
   const StreamSplit sp = stream_split(H, C, p.dyn_units_cap);
   const Share own = share_of(c, H, C, sp);
@@ -676,16 +678,24 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
 // for every dynamic unit u that meets b; warp 0 lists them in shared memory
 // (lanes over CTAs), then each warp merges query heads by their LSE (formula 2
 // of the softmax merge), lane i owning output columns [4i, 4i + 4).
+//
+// The offsets are the scan kernel's output, which has finished by the time this
+// grid launches (the stream kernel signals its dependents only after its own
+// wait on the scan), so the slot list is built while the stream kernel still
+// runs; after the wait only the partials are read, the LSEs and the first
+// kMergeBatch partial rows of a head in one round of independent loads.
+constexpr int kMergeBatch = 8;
+
 __global__ void __launch_bounds__(kMergeWarps * 32) fa_decode_stream_merge_kernel(
     const DecodeParams p) {
   __shared__ int slots[kMaxMergeSlots];
   __shared__ int n_slots_sm;
-  pdl_wait();                                  // the stream kernel's partials
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int xs = p.hb[b], xe = p.hb[b + 1];
+  const int xs = __ldcg(p.hb + b), xe = __ldcg(p.hb + b + 1);
   if (xe <= xs) {                              // no keys (or an invalid length): O = 0, LSE = -inf
+    pdl_wait();
     for (int h = warp; h < p.Hq; h += kMergeWarps) {
       const size_t wid = static_cast<size_t>(b) * p.Hq + h;
       *reinterpret_cast<uint2*>(p.o + wid * kDecD + lane * 4) = make_uint2(0, 0);
@@ -693,7 +703,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) fa_decode_stream_merge_kerne
     }
     return;
   }
-  const int H = p.hb[p.B];
+  const int H = __ldcg(p.hb + p.B);
   const int C = p.nctas;
   const StreamSplit sp = stream_split(H, C, p.dyn_units_cap);
   if (warp == 0) {
@@ -730,39 +740,60 @@ __global__ void __launch_bounds__(kMergeWarps * 32) fa_decode_stream_merge_kerne
   }
   __syncthreads();
   const int ns = n_slots_sm;
+  pdl_wait();                                  // the stream kernel's partials
+  const float4* wo = reinterpret_cast<const float4*>(p.ws_o);
+  auto row = [&](int k, int h) {               // lane's four columns of slot k, head h
+    return __ldcg(wo + (static_cast<size_t>(slots[k]) * p.Hq + h) * (kDecD / 4) + lane);
+  };
   for (int h = warp; h < p.Hq; h += kMergeWarps) {
-    float mx = -INFINITY;
-    for (int k = lane; k < ns; k += 32)
-      mx = fmaxf(mx, p.ws_lse[static_cast<size_t>(slots[k]) * p.Hq + h]);
-#pragma unroll
-    for (int d = 16; d >= 1; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
-    float wsum = 0.f;
+    // 32 slots at a time (one sequence rarely has more): one LSE per lane and the
+    // first kMergeBatch rows load together; a later chunk with a larger maximum
+    // rescales what is accumulated so far
+    float wsum = 0.f, mx = -INFINITY;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (mx > -INFINITY) {
-      // weights lane-parallel, 32 slots at a time; each lane then accumulates its
-      // four columns over those slots with independent loads
-      for (int k0 = 0; k0 < ns; k0 += 32) {
-        float w = 0.f;
-        if (k0 + lane < ns) {
-          const float ls = p.ws_lse[static_cast<size_t>(slots[k0 + lane]) * p.Hq + h];
-          w = (ls == -INFINITY) ? 0.f : ex2((ls - mx) * kLog2e);
+    for (int k0 = 0; k0 < ns; k0 += 32) {
+      const int cnt = min(32, ns - k0);
+      const float ls =
+          lane < cnt ? __ldcg(p.ws_lse + static_cast<size_t>(slots[k0 + lane]) * p.Hq + h)
+                     : -INFINITY;
+      float4 v[kMergeBatch];
+#pragma unroll
+      for (int j = 0; j < kMergeBatch; ++j)
+        if (j < cnt) v[j] = row(k0 + j, h);
+      float m = ls;
+#pragma unroll
+      for (int d = 16; d >= 1; d >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, d));
+      m = fmaxf(m, mx);
+      if (m == -INFINITY) continue;            // every LSE so far is -inf (warp-uniform)
+      const float sc = ex2((mx - m) * kLog2e); // 0 on the first finite chunk
+      acc.x *= sc;
+      acc.y *= sc;
+      acc.z *= sc;
+      acc.w *= sc;
+      wsum *= sc;
+      mx = m;
+      const float w = (ls == -INFINITY) ? 0.f : ex2((ls - mx) * kLog2e);
+      wsum += w;
+      for (int j0 = 0; j0 < cnt; j0 += kMergeBatch) {
+        if (j0 > 0) {
+#pragma unroll
+          for (int j = 0; j < kMergeBatch; ++j)
+            if (j0 + j < cnt) v[j] = row(k0 + j0 + j, h);
         }
-        wsum += w;
-        const int cnt = min(32, ns - k0);
-#pragma unroll 8
-        for (int j = 0; j < cnt; ++j) {
-          const float wj = __shfl_sync(0xffffffffu, w, j);
-          const size_t row = static_cast<size_t>(slots[k0 + j]) * p.Hq + h;
-          const float4 v = reinterpret_cast<const float4*>(p.ws_o + row * kDecD)[lane];
-          acc.x = fmaf(wj, v.x, acc.x);
-          acc.y = fmaf(wj, v.y, acc.y);
-          acc.z = fmaf(wj, v.z, acc.z);
-          acc.w = fmaf(wj, v.w, acc.w);
+#pragma unroll
+        for (int j = 0; j < kMergeBatch; ++j) {
+          const float wj = __shfl_sync(0xffffffffu, w, (j0 + j) & 31);
+          if (j0 + j < cnt) {
+            acc.x = fmaf(wj, v[j].x, acc.x);
+            acc.y = fmaf(wj, v[j].y, acc.y);
+            acc.z = fmaf(wj, v[j].z, acc.z);
+            acc.w = fmaf(wj, v[j].w, acc.w);
+          }
         }
       }
-#pragma unroll
-      for (int d = 16; d >= 1; d >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, d);
     }
+#pragma unroll
+    for (int d = 16; d >= 1; d >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, d);
     const size_t wid = static_cast<size_t>(b) * p.Hq + h;
     const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
     *reinterpret_cast<uint2*>(p.o + wid * kDecD + lane * 4) =
