@@ -64,12 +64,12 @@ static_assert(kRegsProducer * 128 + kRegsConsumer * 256 <= 384 * 168, "register 
 constexpr int kMaxStages = 8;
 constexpr int kStreamSmemBudget = 200 * 1024;
 // Streamed schedule: the half-page list is split into equal contiguous shares,
-// one per CTA.  The first ~90 % of each share is streamed by its own CTA; the
-// last tenth is cut into units of kDynUnit half-pages that go to whichever CTA
+// one per CTA.  The first 15/16 of each share is streamed by its own CTA; the
+// last 16th is cut into units of kDynUnit half-pages that go to whichever CTA
 // asks first, so CTAs that stream more slowly (SMs differ in the bandwidth they
 // get) finish with the others.  Keeping each share's units next to it spreads
 // them over all sequences, so no sequence collects many partials.
-constexpr int kDynDiv = 10;    // 1 / kDynDiv of each share is dynamic
+constexpr int kDynDiv = 16;    // 1 / kDynDiv of each share is dynamic
 constexpr int kDynUnit = 8;    // half-pages per dynamic unit (at least)
 constexpr int kMaxUnitsPerCta = 4;
 constexpr int kMaxStreamCtas = 204;                       // so a sequence has <= 1024 partials
@@ -911,7 +911,7 @@ DecodePlan make_plan(int B, int Hq, int Hkv, int max_pages_per_seq, int nsm) {
     pl.nctas = std::min(nsm, kMaxStreamCtas);
     pl.nstages = kStreamSmemBudget / (2 * stage_kv_bytes(Hkv));
     if (pl.nstages > kMaxStages) pl.nstages = kMaxStages;
-    // enough units for the dynamic tenth of every share of the longest possible list
+    // enough units for the dynamic part of every share of the longest possible list
     const long long h_max = 2LL * B * max_pages_per_seq;
     const long long per_cta = ((h_max + pl.nctas - 1) / pl.nctas) / kDynDiv / kDynUnit + 1;
     pl.dyn_units_cap = static_cast<int>(std::min<long long>(per_cta * pl.nctas, 1 << 24));

@@ -54,9 +54,9 @@ def _short_first(lens):
 
 # (case, block-table width, edit, how the plan fits the 16 MiB array), at 148 SMs:
 CASES = [
-    # persistent schedule, dynamic-unit slots trimmed (888 -> 740), still four per CTA
+    # persistent schedule as fa_decode_paged plans it (592 dynamic-unit slots fit in 740)
     (DECODE_CASES["decode_b64_hq32_hkv8_d128_page16"], None, None),
-    # persistent schedule that fits as fa_decode_paged plans it
+    # persistent schedule that fits as fa_decode_paged plans it, short sequences first
     (DecodeCase("noalloc_small", 5, 16, 2, 128, 16, 1, 900, 400, seed=70), None, _short_first),
     # persistent schedule with the slots trimmed to one dynamic unit per CTA (cap 167)
     (DecodeCase("noalloc_b350", 350, 32, 8, 128, 16, 1, 300, 7200, seed=71), 512, None),
