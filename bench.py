@@ -8,7 +8,10 @@ One step = one pass of the whole path over one batch of synthetic input:
     Hq=32, Hkv=8, D=128, pages of 16 tokens, lengths U[512, 8192], pool of
     40000 pages, bf16).
 Each kernel launch is timed with CUDA events on the launching stream; a 256 MiB
-buffer is written before every launch so no launch finds its inputs in L2.
+buffer is written before every launch so no launch finds its inputs in L2.  The
+decode is also timed (outside the timed region) after a clean flush that reads
+another 256 MiB after the write: the write leaves L2 full of dirty lines whose
+write-back lands inside a bandwidth-bound launch.
 
 ``value`` is prefill TFLOP/s (4*B*Hq*Nq*Nk*D / 2 for causal) summed over ranks
 and divided by the slowest rank's prefill time; the decode KV GB/s is reported
@@ -46,6 +49,7 @@ sys.path.insert(0, ROOT)
 from exact_tiled_attention_40_b200.inputs import (  # noqa: E402
     DECODE_CASES, PAGED_PREFILL_CASES, PREFILL_CASES, VARLEN_CASES, make_decode,
     make_paged_prefill, make_prefill, make_varlen, varlen_flops)
+from exact_tiled_attention_40_b200.l2flush import FLUSH_BYTES, L2Flush  # noqa: E402
 
 METRIC = "attention TFLOP/s & % BF16 tensor peak (prefill); decode KV GB/s & % HBM peak"
 PREFILL = PREFILL_CASES["gqa_b1_hq32_hkv8_n8192_d128_causal"]
@@ -53,7 +57,6 @@ DECODE = DECODE_CASES["decode_b64_hq32_hkv8_d128_page16"]
 RAGGED = VARLEN_CASES["varlen_b16_hq32_hkv8_d128_causal"]
 PAGED = PAGED_PREFILL_CASES["paged_prefill_b16_chunk512_hq32_hkv8_d128"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-FLUSH_BYTES = 256 << 20
 
 
 def dist_env():
@@ -270,7 +273,7 @@ def widened_rows(fa, dev, stream, flush, warmup, steps, peaks, peak_src):
     def timed(launch):
         ts = []
         for i in range(warmup + steps):
-            flush.fill_(i & 0xff)
+            flush(i & 0xff)
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record(stream)
@@ -341,7 +344,7 @@ def fp8_and_backward_rows(fa, dev, stream, flush, warmup, steps, peaks, peak_src
     def timed(launch):
         ts = []
         for i in range(warmup + steps):
-            flush.fill_(i & 0xff)
+            flush(i & 0xff)
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record(stream)
@@ -459,7 +462,7 @@ def dense_prefill_rows(fa, dev, stream, flush, warmup, steps, peaks, peak_src):
             n_warm, n_steps = (3, 5) if long_case else (warmup, steps)
             ts = []
             for i in range(n_warm + n_steps):
-                flush.fill_(i & 0xff)
+                flush(i & 0xff)
                 a = torch.cuda.Event(enable_timing=True)
                 b = torch.cuda.Event(enable_timing=True)
                 a.record(stream)
@@ -571,7 +574,7 @@ def main():
     table, lens = table_h.to(dev), lens_h.to(dev)
     do = torch.empty_like(dq)
     dlse = torch.empty((dcase.B, dcase.Hq), dtype=torch.float32, device=dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
     sum_len = int(lens_h.sum())
@@ -592,11 +595,11 @@ def main():
           for _ in range(args.warmup + args.steps)]
 
     def step(i):
-        flush.fill_(i & 0xff)
+        flush(i & 0xff)
         ev[i][0].record(stream)
         prefill()
         ev[i][1].record(stream)
-        flush.fill_((i + 1) & 0xff)
+        flush((i + 1) & 0xff)
         ev[i][2].record(stream)
         decode()
         ev[i][3].record(stream)
@@ -621,6 +624,19 @@ def main():
     pre_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.warmup, args.warmup + args.steps)]
     dec_ms = [ev[i][2].elapsed_time(ev[i][3]) for i in range(args.warmup, args.warmup + args.steps)]
 
+    # the decode once more, outside the timed region, after a clean flush: the
+    # write-only flush leaves dirty lines whose write-back lands inside each launch
+    ev_c = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            for _ in range(args.warmup + args.steps)]
+    for i in range(args.warmup + args.steps):
+        flush(i, clean=True)
+        ev_c[i][0].record(stream)
+        decode()
+        ev_c[i][1].record(stream)
+    torch.cuda.synchronize()
+    dec_c_ms = [ev_c[i][0].elapsed_time(ev_c[i][1])
+                for i in range(args.warmup, args.warmup + args.steps)]
+
     # ---- end to end through the C ABI with pinned host buffers
     qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
     op = torch.empty(o.shape, dtype=o.dtype).pin_memory()
@@ -632,7 +648,7 @@ def main():
     def e2e_loop(call):
         ts = []
         for i in range(args.warmup + args.steps):
-            flush.fill_(i & 0xff)
+            flush(i & 0xff)
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record(stream)
@@ -707,7 +723,14 @@ def main():
                                 "kernel": "fa_decode_paged call: scan + stream<4> + merge",
                                 "peak_source": f"{peak_src} copy bandwidth",
                                 "frac_of_nominal_8000": dec_achieved / 8000.0},
-                   "ms_per_launch": statistics.mean(dec_ms)},
+                   "ms_per_launch": statistics.mean(dec_ms),
+                   "after_clean_flush": {
+                       "value": kv_bytes / (statistics.mean(dec_c_ms) * 1e-3) / 1e9,
+                       "unit": "GB/s", "ms_per_launch": statistics.mean(dec_c_ms),
+                       "frac_of_measured_copy": dec_bytes / (statistics.mean(dec_c_ms) * 1e-3)
+                       / 1e9 / peaks["hbm_gbs"],
+                       "l2": f"{FLUSH_BYTES >> 20} MiB written, then another "
+                             f"{FLUSH_BYTES >> 20} MiB read: no input and no dirty line left"}},
         "prefill_ms_per_launch": statistics.mean(pre_ms),
         "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "mode": e2e_mode,

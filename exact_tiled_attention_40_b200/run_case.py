@@ -14,7 +14,8 @@ fa_quantize_e4m3 of Q, K and V instead, in GB/s of bf16 read and codes written).
 
 Inputs come from the seeded generator and stay resident on the device; a
 256 MiB buffer is written before every launch so no launch finds its inputs in
-L2.  Each launch is timed with CUDA events on the launching stream.  Handy for
+L2 (--clean-l2 also reads another 256 MiB after it, so that no dirty line of the
+flush is left for the launch to write back: see l2flush.py).  Each launch is timed with CUDA events on the launching stream.  Handy for
 profiling one kernel on one workload.
 """
 from __future__ import annotations
@@ -29,6 +30,7 @@ from . import fa
 from .inputs import (DECODE_CASES, FP8_CASES, PAGED_PREFILL_CASES, PREFILL_CASES, VARLEN_CASES,
                      hadamard_signs, make_decode, make_dout, make_paged_prefill, make_prefill,
                      make_varlen, varlen_flops)
+from .l2flush import L2Flush
 
 
 def main():
@@ -38,9 +40,10 @@ def main():
                     + sorted(PAGED_PREFILL_CASES) + sorted(FP8_CASES))
     ap.add_argument("--op", default="fwd", choices=["fwd", "bwd", "quantize"])
     ap.add_argument("--iters", type=int, default=5)
+    ap.add_argument("--clean-l2", action="store_true")
     args = ap.parse_args()
     dev = torch.device("cuda", 0)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream(dev)
     if args.op == "bwd":
         c = PREFILL_CASES[args.case]
@@ -135,7 +138,7 @@ def main():
         work, unit = int(lens.sum()) * c.Hkv * c.D * 2 * 2 / 1e9, "GB/s"
     times = []
     for i in range(args.iters):
-        flush.fill_(i & 0xff)
+        flush(i, clean=args.clean_l2)
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
